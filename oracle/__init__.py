@@ -1,0 +1,144 @@
+"""fp64 CPU oracle for exact attention, HSTU pointwise attention and the decode step.
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference legs of ``bench.py`` may import this package.  It shares no code with the
+CUDA path and the product never calls it.
+
+The arithmetic lives in ``oracle.c`` (plain C, IEEE double, OpenMP over rows), which materialises each
+score row in full: it is the textbook definition, not a tiled or online computation.  This module only
+marshals numpy/torch arrays into it.  ``build()`` compiles it with gcc.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, -O2, OpenMP, strict IEEE: no -ffast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int)
+        i = ctypes.c_int
+        lib.oracle_attn.restype = ctypes.c_int64
+        lib.oracle_attn.argtypes = [dp, dp, dp, i, i, i, i, ctypes.c_double, i, ip, i, dp, dp]
+        lib.oracle_attn_varlen.restype = ctypes.c_int64
+        lib.oracle_attn_varlen.argtypes = [dp, dp, dp, ip, i, i, i, ctypes.c_double, i, dp, dp]
+        lib.oracle_hstu_jagged.restype = ctypes.c_int64
+        lib.oracle_hstu_jagged.argtypes = [dp, dp, dp, ip, i, i, i, ctypes.c_double, ctypes.c_double, dp]
+        lib.oracle_decode.restype = ctypes.c_int64
+        lib.oracle_decode.argtypes = [dp, dp, dp, ip, i, i, i, i, ctypes.c_double, dp, dp]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_num_threads.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    """Widen a torch tensor (any float dtype, any device) or array to a C-contiguous float64 array."""
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            return np.ascontiguousarray(x.detach().to("cpu", torch.float64).numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _i32(x) -> np.ndarray:
+    try:
+        import torch
+
+        if isinstance(x, torch.Tensor):
+            return np.ascontiguousarray(x.detach().to("cpu", torch.int32).numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+def _dp(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _ip(a):
+    if a is None:
+        return ctypes.POINTER(ctypes.c_int)()
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def attn(q, k, v, scale: float, causal: bool, rows=None, return_flops: bool = False):
+    """Softmax attention of [B,H,N,d] tensors.  Returns (o [B,H,R,d], lse [B,H,R]) as float64 arrays,
+    R = N or len(rows).  ``scale`` is used exactly as given (pass the float32 value the GPU uses)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    assert k.shape == (B, H, N, d) and v.shape == (B, H, N, d)
+    r = None if rows is None else _i32(rows)
+    R = N if r is None else len(r)
+    o = np.zeros((B, H, R, d), np.float64)
+    lse = np.zeros((B, H, R), np.float64)
+    fl = _load().oracle_attn(_dp(q), _dp(k), _dp(v), B, H, N, d, float(scale), int(bool(causal)), _ip(r), R,
+                             _dp(o), _dp(lse))
+    return (o, lse, int(fl)) if return_flops else (o, lse)
+
+
+def attn_varlen(q, k, v, cu_seqlens, scale: float, causal: bool, return_flops: bool = False):
+    """Packed attention: q,k,v [T,H,d], cu_seqlens int [S+1].  Returns (o [T,H,d], lse [T,H])."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cu = _i32(cu_seqlens)
+    T, H, d = q.shape
+    S = len(cu) - 1
+    assert cu[0] == 0 and cu[-1] == T
+    o = np.zeros((T, H, d), np.float64)
+    lse = np.zeros((T, H), np.float64)
+    fl = _load().oracle_attn_varlen(_dp(q), _dp(k), _dp(v), _ip(cu), S, H, d, float(scale), int(bool(causal)),
+                                    _dp(o), _dp(lse))
+    return (o, lse, int(fl)) if return_flops else (o, lse)
+
+
+def hstu_jagged(q, k, v, cu_seqlens, alpha: float, inv_n: float):
+    """HSTU pointwise attention over packed sequences.  Returns o [T,H,d] (float64)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cu = _i32(cu_seqlens)
+    T, H, d = q.shape
+    S = len(cu) - 1
+    assert cu[0] == 0 and cu[-1] == T
+    o = np.zeros((T, H, d), np.float64)
+    _load().oracle_hstu_jagged(_dp(q), _dp(k), _dp(v), _ip(cu), S, H, d, float(alpha), float(inv_n), _dp(o))
+    return o
+
+
+def decode(q, kcache, vcache, kv_lens, scale: float):
+    """Single-query decode: q [B,H,d], caches [B,H,Lmax,d], kv_lens [B].  Returns (o [B,H,d], lse [B,H])."""
+    q, kc, vc = _f64(q), _f64(kcache), _f64(vcache)
+    lens = _i32(kv_lens)
+    B, H, Lmax, d = kc.shape
+    assert q.shape == (B, H, d) and vc.shape == kc.shape and lens.shape == (B,)
+    assert int(lens.max(initial=0)) <= Lmax and int(lens.min(initial=0)) >= 0
+    o = np.zeros((B, H, d), np.float64)
+    lse = np.zeros((B, H), np.float64)
+    _load().oracle_decode(_dp(q), _dp(kc), _dp(vc), _ip(lens), B, H, Lmax, d, float(scale), _dp(o), _dp(lse))
+    return o, lse
