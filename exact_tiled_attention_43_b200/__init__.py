@@ -1,0 +1,209 @@
+"""exact_tiled_attention_43_b200 -- fused exact attention forward passes for B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libeta.so`` (declared in ``include/eta.h``).  Every function
+here only marshals arguments: it checks dtypes/shapes/devices, allocates outputs with torch (device memory
+is torch's job here) and passes raw pointers plus the current CUDA stream to the library, where every step
+of the computation runs in hand-written kernels.  There is no fallback: if ``libeta.so`` is missing or the
+device is not an sm_100 GPU, calls raise.
+
+Entry points (names follow the C ABI):
+  attn_fwd(q, k, v, causal, scale)                     dense [B,H,N,d] softmax attention -> (o, lse)
+  attn_fwd_varlen(q, k, v, cu_seqlens, max_len, ...)   packed [T,H,d] sequences          -> (o, lse)
+  hstu_fwd_jagged(q, k, v, cu_seqlens, max_len, alpha, inv_n)   HSTU pointwise attention -> o
+  attn_decode(q, kcache, vcache, kv_lens, scale)       one-query decode over a KV cache  -> (o, lse)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libeta.so")
+_lib = None
+
+ETA_OUT_BF16, ETA_OUT_F32 = 0, 1
+ETA_DEV_OK, ETA_DEV_TIMEOUT, ETA_DEV_BAD_KVLEN, ETA_DEV_BAD_CUSEQ = 0, 1, 2, 3
+
+# name -> (restype, argtypes); mirrors include/eta.h
+_VP, _I, _F, _SZ, _LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_longlong
+SIGNATURES = {
+    "attn_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "attn_fwd_varlen": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "hstu_fwd_jagged": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _F, _VP]),
+    "attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "attn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _SZ, _VP]),
+    "eta_status": (_I, [_VP]),
+    "eta_strerror": (ctypes.c_char_p, [_I]),
+    "eta_set_wait_timeout_ns": (None, [_LL]),
+    "eta_selftest_wait_timeout": (_I, [_VP]),
+}
+
+
+class EtaError(RuntimeError):
+    pass
+
+
+def lib():
+    """Loads libeta.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise EtaError(f"{LIB_PATH} is missing: build it with `python -m exact_tiled_attention_43_b200.build` "
+                           "(or __graft_entry__.build()); there is no fallback implementation")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().eta_strerror(int(code)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise EtaError(f"{what} failed: {strerror(rc)} (code {rc})")
+
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _stream_ptr(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _need(t, name, dtype, ndim):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def default_scale(d: int) -> float:
+    """The float32 value of 1/sqrt(d)."""
+    import numpy as np
+
+    return float(np.float32(1.0 / math.sqrt(d)))
+
+
+def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out_dtype=None, out=None, lse=None,
+             return_lse: bool = True, stream=None):
+    """Dense exact attention: q, k, v bf16 [B,H,N,d].  Returns (o [B,H,N,d], lse fp32 [B,H,N] or None)."""
+    torch = _torch()
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 4)
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape")
+    out_dtype = out_dtype or torch.bfloat16
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=out_dtype, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    scale = default_scale(d) if scale is None else float(scale)
+    odt = ETA_OUT_F32 if out.dtype == torch.float32 else ETA_OUT_BF16
+    rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse if return_lse else None), B, H, N, d, scale,
+                        int(bool(causal)), odt, _stream_ptr(stream))
+    _check(rc, "attn_fwd")
+    return out, (lse if return_lse else None)
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens, max_len: int, causal: bool = False, scale: float | None = None,
+                    out_dtype=None, return_lse: bool = True, stream=None):
+    """Packed exact attention: q, k, v bf16 [T,H,d], cu_seqlens int32 [S+1] (device).
+    Returns (o [T,H,d], lse fp32 [T,H] or None)."""
+    torch = _torch()
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    T, H, d = q.shape
+    out = torch.empty((T, H, d), dtype=out_dtype or torch.bfloat16, device=q.device)
+    lse = torch.empty((T, H), dtype=torch.float32, device=q.device) if return_lse else None
+    scale = default_scale(d) if scale is None else float(scale)
+    odt = ETA_OUT_F32 if out.dtype == torch.float32 else ETA_OUT_BF16
+    rc = lib().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens),
+                               cu_seqlens.numel() - 1, int(max_len), T, H, d, scale, int(bool(causal)), odt,
+                               _stream_ptr(stream))
+    _check(rc, "attn_fwd_varlen")
+    return out, lse
+
+
+def hstu_fwd_jagged(q, k, v, cu_seqlens, max_len: int, alpha: float, inv_n: float, out=None, stream=None):
+    """HSTU pointwise attention over packed sequences: q, k, v bf16 [T,H,d] -> o bf16 [T,H,d]."""
+    torch = _torch()
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, torch.bfloat16, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    T, H, d = q.shape
+    if out is None:
+        out = torch.empty((T, H, d), dtype=torch.bfloat16, device=q.device)
+    rc = lib().hstu_fwd_jagged(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                               int(max_len), T, H, d, float(alpha), float(inv_n), _stream_ptr(stream))
+    _check(rc, "hstu_fwd_jagged")
+    return out
+
+
+def attn_decode_workspace_size(B: int, H: int, Lmax: int, d: int) -> int:
+    return int(lib().attn_decode_workspace_size(B, H, Lmax, d))
+
+
+def attn_decode(q, kcache, vcache, kv_lens, scale: float | None = None, workspace=None, out=None, lse=None,
+                stream=None):
+    """One decode step: q bf16 [B,H,d], caches bf16 [B,H,Lmax,d], kv_lens int32 [B] (device).
+    Returns (o bf16 [B,H,d], lse fp32 [B,H])."""
+    torch = _torch()
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kcache, "kcache", torch.bfloat16, 4)
+    _need(vcache, "vcache", torch.bfloat16, 4)
+    _need(kv_lens, "kv_lens", torch.int32, 1)
+    B, H, Lmax, d = kcache.shape
+    if vcache.shape != kcache.shape or q.shape != (B, H, d) or kv_lens.shape != (B,):
+        raise ValueError("inconsistent decode shapes")
+    need = attn_decode_workspace_size(B, H, Lmax, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    scale = default_scale(d) if scale is None else float(scale)
+    rc = lib().attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kv_lens), _ptr(out), _ptr(lse), B, H, Lmax, d,
+                           scale, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check(rc, "attn_decode")
+    return out, lse
+
+
+def status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status word (ETA_DEV_*)."""
+    rc = lib().eta_status(_stream_ptr(stream))
+    if rc < 0:
+        raise EtaError(f"eta_status failed: {strerror(rc)}")
+    return rc
+
+
+def set_wait_timeout_ns(ns: int):
+    lib().eta_set_wait_timeout_ns(int(ns))
+
+
+def selftest_wait_timeout(stream=None):
+    _check(lib().eta_selftest_wait_timeout(_stream_ptr(stream)), "eta_selftest_wait_timeout")

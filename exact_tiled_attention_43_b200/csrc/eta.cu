@@ -1,0 +1,292 @@
+// eta.cu -- the C ABI of libeta.so (declared in include/eta.h): argument validation, TMA tensor-map
+// encoding, kernel launches and the device status word.  The kernels themselves live in prefill.cuh and
+// decode.cuh and are compiled into this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "eta.h"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace {
+
+constexpr long long kDefaultWaitNs = 2000000000LL;  // 2 s
+long long g_wait_ns = kDefaultWaitNs;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The current device must be sm_100 (B200 class).  Cached per device ordinal.
+int check_device() {
+  static int cache[64];  // 0 unknown, 1 ok, -1 bad
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ETA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return ETA_ERR_DEVICE;
+  if (cache[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return ETA_ERR_CUDA;
+    cache[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return cache[dev] == 1 ? ETA_OK : ETA_ERR_DEVICE;
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no -lcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// bf16 rows of `d` elements; box = 64 elements (128 B, one swizzle span) x 128 rows.
+// dense  : tensor [BH][N][d]      -> dims {d, N, BH},  box {64, 128, 1}
+// packed : tensor [T][H][d]       -> dims {d, H, T},   box {64, 1, 128}
+int encode_map(CUtensorMap *m, const void *base, bool packed, long long n1, long long n2, int d) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return ETA_ERR_CUDA;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3], estr[3] = {1, 1, 1};
+  dims[0] = (cuuint64_t)d;
+  if (packed) {  // n1 = H, n2 = T
+    dims[1] = (cuuint64_t)n1;
+    dims[2] = (cuuint64_t)n2;
+    strides[0] = (cuuint64_t)d * 2;
+    strides[1] = (cuuint64_t)n1 * d * 2;
+    box[0] = 64; box[1] = 1; box[2] = 128;
+  } else {       // n1 = N, n2 = BH
+    dims[1] = (cuuint64_t)n1;
+    dims[2] = (cuuint64_t)n2;
+    strides[0] = (cuuint64_t)d * 2;
+    strides[1] = (cuuint64_t)n1 * d * 2;
+    box[0] = 64; box[1] = 128; box[2] = 1;
+  }
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ETA_OK : ETA_ERR_CUDA;
+}
+
+template <int D, int MODE>
+int launch_prefill(const void *q, const void *k, const void *v, bool packed, long long n1, long long n2, dim3 grid,
+                   const eta::PrefillParams &p, cudaStream_t stream) {
+  CUtensorMap mq, mk, mv;
+  int rc;
+  if ((rc = encode_map(&mq, q, packed, n1, n2, D)) != ETA_OK) return rc;
+  if ((rc = encode_map(&mk, k, packed, n1, n2, D)) != ETA_OK) return rc;
+  if ((rc = encode_map(&mv, v, packed, n1, n2, D)) != ETA_OK) return rc;
+  auto kern = eta::prefill_kernel<D, MODE>;
+  constexpr int smem = eta::PfCfg<D>::SMEM_BYTES;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ETA_ERR_CUDA;
+  kern<<<grid, eta::PF_THREADS, smem, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
+}
+
+bool finite_pos(float x) { return std::isfinite(x) && x > 0.f; }
+
+int prefill_common(int mode, const void *q, const void *k, const void *v, void *o, float *lse,
+                   const int *cu_seqlens, int B, int S, int N, int max_len, int T_total, int H, int d,
+                   float scale, int causal, int o_dtype, float alpha, float inv_n, void *stream) {
+  if (!q || !k || !v || !o) return ETA_ERR_NULL;
+  if (mode != eta::MODE_DENSE && !cu_seqlens) return ETA_ERR_NULL;
+  if (d != 64 && d != 128) return ETA_ERR_HEAD_DIM;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ETA_ERR_ALIGN;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ETA_ERR_ALIGN;
+  if (o_dtype != ETA_OUT_BF16 && o_dtype != ETA_OUT_F32) return ETA_ERR_ARG;
+  if (causal != 0 && causal != 1) return ETA_ERR_ARG;
+  if (H <= 0 || H > 65535) return ETA_ERR_SHAPE;
+  eta::PrefillParams p{};
+  dim3 grid;
+  long long n1, n2;
+  if (mode == eta::MODE_DENSE) {
+    if (B <= 0 || N <= 0) return ETA_ERR_SHAPE;
+    const long long bh = (long long)B * H;
+    const long long nblk = ((long long)N + 255) / 256;
+    if (bh > INT_MAX || nblk > 65535) return ETA_ERR_SHAPE;
+    grid = dim3((unsigned)bh, (unsigned)nblk, 1);
+    n1 = N;
+    n2 = bh;
+    p.N = N;
+  } else {
+    if (S <= 0 || max_len <= 0 || T_total < 0 || S > 65535) return ETA_ERR_SHAPE;
+    if (T_total == 0) return ETA_OK;  // nothing to compute
+    const long long nblk = ((long long)max_len + 255) / 256;
+    if (nblk > 65535) return ETA_ERR_SHAPE;
+    grid = dim3((unsigned)H, (unsigned)nblk, (unsigned)S);
+    n1 = H;
+    n2 = T_total;
+    p.max_len = max_len;
+  }
+  if (mode == eta::MODE_HSTU) {
+    if (!std::isfinite(alpha) || !finite_pos(inv_n)) return ETA_ERR_ARG;
+    if (o_dtype != ETA_OUT_BF16) return ETA_ERR_ARG;
+  } else if (!finite_pos(scale)) {
+    return ETA_ERR_ARG;
+  }
+  int rc = check_device();
+  if (rc != ETA_OK) return rc;
+  p.o = o;
+  p.lse = (mode == eta::MODE_HSTU) ? nullptr : lse;
+  p.cu_seqlens = cu_seqlens;
+  p.H = H;
+  p.causal = causal;
+  p.o_f32 = (o_dtype == ETA_OUT_F32);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.hstu_half_alpha = 0.5f * alpha;
+  p.hstu_out = 0.5f * alpha * inv_n;
+  p.wait_ns = g_wait_ns;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool packed = (mode != eta::MODE_DENSE);
+  if (d == 64) {
+    if (mode == eta::MODE_DENSE) return launch_prefill<64, eta::MODE_DENSE>(q, k, v, packed, n1, n2, grid, p, st);
+    if (mode == eta::MODE_VARLEN) return launch_prefill<64, eta::MODE_VARLEN>(q, k, v, packed, n1, n2, grid, p, st);
+    return launch_prefill<64, eta::MODE_HSTU>(q, k, v, packed, n1, n2, grid, p, st);
+  }
+  if (mode == eta::MODE_DENSE) return launch_prefill<128, eta::MODE_DENSE>(q, k, v, packed, n1, n2, grid, p, st);
+  if (mode == eta::MODE_VARLEN) return launch_prefill<128, eta::MODE_VARLEN>(q, k, v, packed, n1, n2, grid, p, st);
+  return launch_prefill<128, eta::MODE_HSTU>(q, k, v, packed, n1, n2, grid, p, st);
+}
+
+template <int D>
+int launch_decode(const eta::DecodeParams &p, cudaStream_t st) {
+  constexpr int smem = 2 * eta::DEC_STAGES * eta::DEC_ROWS * D * 2;
+  auto ks = eta::decode_split_kernel<D>;
+  if (cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return ETA_ERR_CUDA;
+  ks<<<dim3(p.max_splits, p.H, p.B), eta::DEC_THREADS, smem, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ETA_ERR_CUDA;
+  eta::decode_combine_kernel<D><<<dim3(p.H, p.B), D, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
+}
+
+size_t decode_ws_bytes(int B, int H, int Lmax, int d) {
+  const size_t n = (size_t)B * H * eta::decode_max_splits(Lmax);
+  const size_t o_bytes = (n * d * sizeof(float) + 255) & ~size_t(255);
+  return o_bytes + n * sizeof(float);
+}
+
+__global__ void selftest_wait_kernel(long long wait_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    eta::mbar_init(&bar, 1);  // nothing ever arrives
+    abort_flag = 0;
+    eta::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) eta::mbar_wait(&bar, 0, &abort_flag, wait_ns);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
+             float scale, int causal, int o_dtype, void *stream) {
+  return prefill_common(eta::MODE_DENSE, q, k, v, o, lse, nullptr, B, 0, N, 0, 0, H, d, scale, causal, o_dtype, 0.f,
+                        1.f, stream);
+}
+
+int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse, const int *cu_seqlens, int S,
+                    int max_len, int T_total, int H, int d, float scale, int causal, int o_dtype, void *stream) {
+  return prefill_common(eta::MODE_VARLEN, q, k, v, o, lse, cu_seqlens, 0, S, 0, max_len, T_total, H, d, scale, causal,
+                        o_dtype, 0.f, 1.f, stream);
+}
+
+int hstu_fwd_jagged(const void *q, const void *k, const void *v, void *o, const int *cu_seqlens, int S, int max_len,
+                    int T_total, int H, int d, float alpha, float inv_n, void *stream) {
+  return prefill_common(eta::MODE_HSTU, q, k, v, o, nullptr, cu_seqlens, 0, S, 0, max_len, T_total, H, d, 1.f, 1,
+                        ETA_OUT_BF16, alpha, inv_n, stream);
+}
+
+size_t attn_decode_workspace_size(int B, int H, int Lmax, int d) {
+  if (B <= 0 || H <= 0 || Lmax <= 0 || (d != 64 && d != 128)) return 0;
+  return decode_ws_bytes(B, H, Lmax, d);
+}
+
+int attn_decode(const void *q, const void *kcache, const void *vcache, const int *kv_lens, void *o, float *lse, int B,
+                int H, int Lmax, int d, float scale, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!q || !kcache || !vcache || !kv_lens || !o || !workspace) return ETA_ERR_NULL;
+  if (d != 64 && d != 128) return ETA_ERR_HEAD_DIM;
+  if (B <= 0 || H <= 0 || Lmax <= 0 || B > 65535 || H > 65535) return ETA_ERR_SHAPE;
+  if ((long long)B * H * Lmax * d >= (1LL << 40)) return ETA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o) || !aligned16(workspace))
+    return ETA_ERR_ALIGN;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ETA_ERR_ALIGN;
+  if (!finite_pos(scale)) return ETA_ERR_ARG;
+  if (workspace_bytes < decode_ws_bytes(B, H, Lmax, d)) return ETA_ERR_WORKSPACE;
+  int rc = check_device();
+  if (rc != ETA_OK) return rc;
+  eta::DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.kc = static_cast<const __nv_bfloat16 *>(kcache);
+  p.vc = static_cast<const __nv_bfloat16 *>(vcache);
+  p.kv_lens = kv_lens;
+  p.o = static_cast<__nv_bfloat16 *>(o);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Lmax = Lmax;
+  p.chunk = eta::decode_chunk(Lmax);
+  p.max_splits = eta::decode_max_splits(Lmax);
+  const size_t n = (size_t)B * H * p.max_splits;
+  p.part_o = static_cast<float *>(workspace);
+  p.part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + ((n * d * sizeof(float) + 255) & ~size_t(255)));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_ns = g_wait_ns;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_decode<64>(p, st) : launch_decode<128>(p, st);
+}
+
+int eta_status(void *stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ETA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, eta::g_status, sizeof(int)) != cudaSuccess) return ETA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(eta::g_status, &zero, sizeof(int)) != cudaSuccess) return ETA_ERR_CUDA;
+  return v;
+}
+
+const char *eta_strerror(int code) {
+  switch (code) {
+    case ETA_OK: return "ok";
+    case ETA_ERR_NULL: return "a required pointer is NULL";
+    case ETA_ERR_HEAD_DIM: return "head dimension must be 64 or 128";
+    case ETA_ERR_SHAPE: return "a size is out of range or inconsistent";
+    case ETA_ERR_ALIGN: return "a tensor pointer is not 16-byte aligned";
+    case ETA_ERR_WORKSPACE: return "workspace is smaller than attn_decode_workspace_size()";
+    case ETA_ERR_CUDA: return "a CUDA call or kernel launch failed";
+    case ETA_ERR_ARG: return "a flag or scalar argument is out of range";
+    case ETA_ERR_DEVICE: return "the current device is not an sm_100 GPU";
+    case ETA_DEV_TIMEOUT: return "device: a bounded pipeline wait expired";
+    case ETA_DEV_BAD_KVLEN: return "device: kv_lens entry outside [0, Lmax]";
+    case ETA_DEV_BAD_CUSEQ: return "device: cu_seqlens decreasing or a sequence longer than max_len";
+    default: return "unknown code";
+  }
+}
+
+void eta_set_wait_timeout_ns(long long ns) { g_wait_ns = ns > 0 ? ns : kDefaultWaitNs; }
+
+int eta_selftest_wait_timeout(void *stream) {
+  int rc = check_device();
+  if (rc != ETA_OK) return rc;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_wait_ns);
+  return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
+}
+
+}  // extern "C"

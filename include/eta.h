@@ -1,0 +1,165 @@
+/*
+ * eta.h -- C ABI of libeta.so: fused, IO-aware exact attention forward passes for NVIDIA B200 (sm_100a).
+ *
+ * Every entry point computes one of the operations the reference pages define, tile by tile on the GPU,
+ * without ever writing the n x n score matrix to HBM:
+ *
+ *   attn_fwd / attn_fwd_varlen   O = softmax(scale * Q K^T [+ causal mask]) V, plus the row logsumexp.
+ *       "FlashAttention (TH)", section "ปัญหาของ Attention แบบมาตรฐาน" (the formula) and section
+ *       "การคำนวณ Softmax แบบออนไลน์" (running max and exp-sum); "CANN ops-transformer 的 FlashAttention：
+ *       把大模型的记忆从 32GB 压到 8GB，怎么做到的", section "FlashAttention 的解法" (online softmax, steps 1-4,
+ *       only the final output written back).
+ *   hstu_fwd_jagged              O = (SiLU(alpha * Q K^T) * causal_mask / n) V over packed sequences.
+ *       "同样是Attention架构，为什么昇腾NPU跑HSTU时延降低10倍、显存省97%？", section "先搞懂：HSTU到底难在哪？"
+ *       (the definition), "绝杀优化二：内置Mask生成" (mask generated in-kernel, masked tiles skipped) and
+ *       "绝杀优化三：Jagged变长张量" (packed values + per-sequence lengths, no padding).
+ *   attn_decode                  one new query per (batch, head) against a long KV cache.
+ *       "AI attention complexity ledger", section "带宽账：decode 阶段的真正瓶颈"
+ *       (s_j = q . k_j over all cached keys, o = sum_j p_j v_j; HBM-bound).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers named q, k, v, o, kcache, vcache, lse, cu_seqlens, kv_lens, workspace are DEVICE pointers
+ *    (cudaMalloc'd or equivalent) on the current CUDA device.  The caller owns every buffer; the library
+ *    allocates no device memory and keeps no per-call state.
+ *  - bf16 means IEEE bfloat16 stored as 16-bit words; all tensors are contiguous, row-major, with the
+ *    layouts given per call.  q, k, v, o and the caches must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only enqueues work on it and
+ *    returns; results are ready when the stream reaches that point.
+ *  - Return value: 0 (ETA_OK) when the work was enqueued, a negative ETA_ERR_* code when the arguments
+ *    are rejected on the host (nothing is enqueued then) or a CUDA launch failed.
+ *  - Conditions only the device can see (a kv_lens entry outside [0, Lmax], cu_seqlens that decrease or
+ *    hold a sequence longer than max_len, a pipeline wait that ran out of time) never trap: the kernel
+ *    keeps every access in bounds, records the first such condition in a device status word and carries
+ *    on or returns.  Read it with eta_status().
+ *  - Head dimension d must be 64 or 128.  The arithmetic is bf16 x bf16 products accumulated in fp32
+ *    (tensor cores); softmax statistics and lse are fp32.
+ */
+#ifndef ETA_H_
+#define ETA_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define ETA_API __attribute__((visibility("default")))
+#else
+#define ETA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host-side error codes (negative) returned by the entry points. */
+#define ETA_OK 0
+#define ETA_ERR_NULL (-1)      /* a required pointer is NULL */
+#define ETA_ERR_HEAD_DIM (-2)  /* d is not 64 or 128 */
+#define ETA_ERR_SHAPE (-3)     /* a size is <= 0, too large for 32-bit indexing, or inconsistent */
+#define ETA_ERR_ALIGN (-4)     /* a tensor pointer is not 16-byte aligned */
+#define ETA_ERR_WORKSPACE (-5) /* workspace smaller than attn_decode_workspace_size() */
+#define ETA_ERR_CUDA (-6)      /* a CUDA runtime/driver call or a kernel launch failed */
+#define ETA_ERR_ARG (-7)       /* a flag or scalar is out of range (o_dtype, scale, alpha, inv_n ...) */
+#define ETA_ERR_DEVICE (-8)    /* the current device is not an sm_100 (B200-class) GPU */
+
+/* Device status codes (positive) returned by eta_status(). */
+#define ETA_DEV_OK 0
+#define ETA_DEV_TIMEOUT 1     /* a bounded pipeline wait expired; the kernel abandoned its tile */
+#define ETA_DEV_BAD_KVLEN 2   /* attn_decode: kv_lens[b] < 0 or > Lmax (clamped into range) */
+#define ETA_DEV_BAD_CUSEQ 3   /* varlen/jagged: cu_seqlens decreasing or a sequence longer than max_len */
+
+/* Output element type selector for attn_fwd / attn_fwd_varlen. */
+#define ETA_OUT_BF16 0
+#define ETA_OUT_F32 1
+
+/*
+ * attn_fwd -- dense multi-head exact attention forward.
+ *   q, k, v : bf16 [B, H, N, d]   (batch, heads, sequence, head dim; the pages' [batch, heads, seq_len,
+ *                                  head_dim] layout, "ai6s.net FlashAttention" page, usage example)
+ *   o       : [B, H, N, d], bf16 (o_dtype = ETA_OUT_BF16) or fp32 (ETA_OUT_F32)
+ *   lse     : fp32 [B, H, N], natural-log logsumexp of the scaled score row, m_i + ln(sum_j e^(s_ij - m_i));
+ *             may be NULL (not written)
+ *   scale   : multiplies Q K^T before the softmax (1/sqrt(d) in the formula); finite and > 0
+ *   causal  : 0 = every key; 1 = query i sees keys j <= i (top-left aligned, diagonal included)
+ * Errors: ETA_ERR_NULL, ETA_ERR_HEAD_DIM, ETA_ERR_SHAPE (B,H,N <= 0 or B*H*N*d >= 2^31), ETA_ERR_ALIGN,
+ *         ETA_ERR_ARG, ETA_ERR_DEVICE, ETA_ERR_CUDA.
+ */
+ETA_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
+             float scale, int causal, int o_dtype, void *stream);
+
+/*
+ * attn_fwd_varlen -- exact attention over S packed sequences (no padding).
+ *   q, k, v    : bf16 [T, H, d], T = cu_seqlens[S]; sequence s owns rows cu_seqlens[s] .. cu_seqlens[s+1]-1
+ *   o          : [T, H, d] bf16 or fp32 (o_dtype);  lse: fp32 [T, H] or NULL
+ *   cu_seqlens : int32 [S+1], device; cu_seqlens[0] = 0, non-decreasing
+ *   max_len    : an upper bound on every sequence length (sizes the launch); T_total : cu_seqlens[S]
+ *                as known to the host (used to size tensor maps; must match the device value)
+ *   No query attends across a sequence boundary; causal is per sequence (local indices).
+ * Zero-length sequences produce nothing.  Errors as attn_fwd, plus device status ETA_DEV_BAD_CUSEQ.
+ */
+ETA_API int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse, const int *cu_seqlens,
+                    int S, int max_len, int T_total, int H, int d, float scale, int causal, int o_dtype,
+                    void *stream);
+
+/*
+ * hstu_fwd_jagged -- HSTU pointwise attention over S packed sequences:
+ *   x_ij = alpha * q_i . k_j ;  p_ij = silu(x_ij) * inv_n  for j <= i (local indices), 0 otherwise ;
+ *   o_i = sum_j p_ij v_j.
+ *   q, k, v : bf16 [T, H, d]; o : bf16 [T, H, d]; cu_seqlens, S, max_len, T_total as attn_fwd_varlen.
+ *   alpha   : the page's alpha (finite); inv_n : 1/n of the page's "x *= mask / n" (finite, > 0).
+ * There is no softmax, no running max and no lse.  Errors as attn_fwd_varlen.
+ */
+ETA_API int hstu_fwd_jagged(const void *q, const void *k, const void *v, void *o, const int *cu_seqlens, int S,
+                    int max_len, int T_total, int H, int d, float alpha, float inv_n, void *stream);
+
+/*
+ * attn_decode_workspace_size -- bytes of device workspace attn_decode needs for these sizes
+ * (split-KV partial outputs and their logsumexps).  Returns 0 for invalid sizes.
+ */
+ETA_API size_t attn_decode_workspace_size(int B, int H, int Lmax, int d);
+
+/*
+ * attn_decode -- one decode step: for each (b, h), the single query q[b,h,:] attends (non-causally) to the
+ * cached keys/values rows 0 .. kv_lens[b]-1.
+ *   q         : bf16 [B, H, d]
+ *   kcache    : bf16 [B, H, Lmax, d];  vcache : bf16 [B, H, Lmax, d]; rows >= kv_lens[b] are never read
+ *   kv_lens   : int32 [B], device, each in [0, Lmax]; a zero length gives o = 0, lse = -inf
+ *   o         : bf16 [B, H, d];  lse : fp32 [B, H] or NULL
+ *   workspace : device buffer of at least attn_decode_workspace_size(B, H, Lmax, d) bytes, 16-byte
+ *               aligned, owned by the caller; its contents need no initialisation and are scratch.
+ * The cache is split along the sequence into chunks processed by independent CTAs (split-KV); the chunks'
+ * partial results are merged with logsumexp weights, which is exact.
+ * Errors as attn_fwd, plus ETA_ERR_WORKSPACE and device status ETA_DEV_BAD_KVLEN.
+ */
+ETA_API int attn_decode(const void *q, const void *kcache, const void *vcache, const int *kv_lens, void *o, float *lse,
+                int B, int H, int Lmax, int d, float scale, void *workspace, size_t workspace_bytes,
+                void *stream);
+
+/*
+ * eta_status -- synchronises `stream`, returns the device status word of the current device
+ * (ETA_DEV_*; the first condition recorded since the last call) and clears it.  Returns ETA_ERR_CUDA if
+ * the synchronisation or the copy failed.
+ */
+ETA_API int eta_status(void *stream);
+
+/* eta_strerror -- a static, human-readable description of any ETA_* code. */
+ETA_API const char *eta_strerror(int code);
+
+/*
+ * eta_set_wait_timeout_ns -- upper bound, in nanoseconds of %globaltimer, on every pipeline wait inside
+ * the kernels (default 2e9 = 2 s).  A wait that runs out records ETA_DEV_TIMEOUT and the kernel returns.
+ * Values <= 0 restore the default.  Applies to launches made after the call.
+ */
+ETA_API void eta_set_wait_timeout_ns(long long ns);
+
+/*
+ * eta_selftest_wait_timeout -- launches one CTA that waits on a pipeline barrier nothing will ever
+ * complete, under the current bounded-wait limit, so that a test can check the limit and the status word
+ * without faulting or hanging the GPU.  Returns 0 when enqueued; the caller then reads eta_status().
+ */
+ETA_API int eta_selftest_wait_timeout(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ETA_H_ */

@@ -1,0 +1,81 @@
+"""The C ABI library loads, exports every entry point include/eta.h declares, and rejects bad arguments
+on the host before touching any device (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import __graft_entry__  # noqa: F401  (makes sure the build entry exists)
+import exact_tiled_attention_43_b200 as eta
+from exact_tiled_attention_43_b200 import build as eta_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    eta_build.build()
+    return eta.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "eta.h")).read()
+    return re.findall(r"^ETA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src, flags=re.M)
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/eta.h but not exported by libeta.so"
+        assert n in eta.SIGNATURES, f"{n} has no Python binding signature"
+
+
+def test_strerror_covers_codes(L):
+    for c in range(-8, 4):
+        assert eta.strerror(c) != "unknown code"
+    assert eta.strerror(12345) == "unknown code"
+
+
+A = ctypes.c_void_p(0x10000)      # a 16-byte aligned, never dereferenced address
+MIS = ctypes.c_void_p(0x10008)    # misaligned
+NUL = ctypes.c_void_p(0)
+S = ctypes.c_void_p(0)
+
+
+def test_attn_fwd_host_validation(L):
+    assert L.attn_fwd(NUL, A, A, A, NUL, 1, 1, 128, 64, 0.125, 0, 0, S) == -1
+    assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 96, 0.125, 0, 0, S) == -2
+    assert L.attn_fwd(A, A, A, A, NUL, 0, 1, 128, 64, 0.125, 0, 0, S) == -3
+    assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 0, 64, 0.125, 0, 0, S) == -3
+    assert L.attn_fwd(A, A, MIS, A, NUL, 1, 1, 128, 64, 0.125, 0, 0, S) == -4
+    assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 64, 0.125, 0, 7, S) == -7
+    assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 64, float("nan"), 0, 0, S) == -7
+    assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 64, -1.0, 0, 0, S) == -7
+    assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 64, 0.125, 2, 0, S) == -7
+    # valid arguments without a usable GPU: a clean negative code, no crash
+    rc = L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 64, 0.125, 0, 0, S)
+    assert rc in (-6, -8)
+
+
+def test_varlen_and_hstu_host_validation(L):
+    assert L.attn_fwd_varlen(A, A, A, A, NUL, NUL, 2, 128, 256, 1, 64, 0.125, 1, 0, S) == -1
+    assert L.attn_fwd_varlen(A, A, A, A, NUL, A, 0, 128, 256, 1, 64, 0.125, 1, 0, S) == -3
+    assert L.attn_fwd_varlen(A, A, A, A, NUL, A, 2, 0, 256, 1, 64, 0.125, 1, 0, S) == -3
+    assert L.attn_fwd_varlen(A, A, A, A, NUL, A, 2, 128, 0, 1, 64, 0.125, 1, 0, S) == 0  # empty batch: no work
+    assert L.hstu_fwd_jagged(A, A, A, A, A, 2, 128, 256, 1, 64, 0.125, 0.0, S) == -7
+    assert L.hstu_fwd_jagged(A, A, A, A, A, 2, 128, 256, 1, 64, float("inf"), 1.0, S) == -7
+    assert L.hstu_fwd_jagged(A, A, A, MIS, A, 2, 128, 256, 1, 64, 0.125, 1.0, S) == -4
+    assert L.hstu_fwd_jagged(A, A, A, A, A, 2, 128, 256, 1, 32, 0.125, 1.0, S) == -2
+
+
+def test_decode_host_validation(L):
+    ws = eta.attn_decode_workspace_size(64, 32, 32768, 128)
+    assert ws > 0 and eta.attn_decode_workspace_size(0, 32, 100, 128) == 0
+    assert eta.attn_decode_workspace_size(1, 1, 100, 96) == 0
+    assert L.attn_decode(A, A, A, A, A, NUL, 64, 32, 32768, 128, 0.088, A, ws - 1, S) == -5
+    assert L.attn_decode(A, A, A, NUL, A, NUL, 64, 32, 32768, 128, 0.088, A, ws, S) == -1
+    assert L.attn_decode(A, A, A, A, A, NUL, 64, 32, 32768, 100, 0.088, A, ws, S) == -2
+    assert L.attn_decode(A, MIS, A, A, A, NUL, 64, 32, 32768, 128, 0.088, A, ws, S) == -4
+    assert L.attn_decode(A, A, A, A, A, NUL, 64, 32, 32768, 128, 0.0, A, ws, S) == -7

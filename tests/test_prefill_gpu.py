@@ -1,0 +1,111 @@
+"""attn_fwd (dense prefill) against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import exact_tiled_attention_43_b200 as eta
+import oracle
+from exact_tiled_attention_43_b200 import inputs
+from parity import check_lse, check_o
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_tiny_config(causal, out_dtype):
+    """B=1, H=2, N=256, d=64, every output element compared."""
+    q, k, v = (t.to(DEV) for t in inputs.dense_qkv(inputs.TINY, 1, 2, 256, 64))
+    scale = eta.default_scale(64)
+    o, lse = eta.attn_fwd(q, k, v, causal=causal, scale=scale, out_dtype=out_dtype)
+    assert eta.status() == 0
+    o_ref, lse_ref = oracle.attn(q, k, v, scale, causal)
+    check_o(o, o_ref, f"tiny causal={causal}")
+    check_lse(lse, lse_ref, "tiny lse")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 2, 17, 127, 128, 129, 255, 256, 257, 700])
+def test_ragged_lengths(d, causal, N):
+    B, H = 2, 3
+    q, k, v = (t.to(DEV) for t in inputs.dense_qkv(7, B, H, N, d))
+    scale = eta.default_scale(d)
+    o, lse = eta.attn_fwd(q, k, v, causal=causal, scale=scale)
+    assert eta.status() == 0
+    o_ref, lse_ref = oracle.attn(q, k, v, scale, causal)
+    check_o(o, o_ref, f"N={N} d={d} causal={causal}")
+    check_lse(lse, lse_ref, "lse")
+
+
+def test_no_lse_and_custom_scale():
+    q, k, v = (t.to(DEV) for t in inputs.dense_qkv(8, 1, 2, 300, 128))
+    o, none = eta.attn_fwd(q, k, v, causal=True, scale=0.05, return_lse=False)
+    assert none is None
+    o_ref, _ = oracle.attn(q, k, v, 0.05, True)
+    check_o(o, o_ref, "scale=0.05")
+
+
+def test_large_score_magnitudes():
+    """Scaled scores of order 1e2 exercise the running-max rescale path (and its threshold)."""
+    q, k, v = (t.to(DEV) for t in inputs.dense_qkv(9, 1, 2, 640, 64))
+    q = (q.float() * 8).to(torch.bfloat16)
+    k = (k.float() * 4).to(torch.bfloat16)
+    for causal in (False, True):
+        o, lse = eta.attn_fwd(q, k, v, causal=causal)
+        o_ref, lse_ref = oracle.attn(q, k, v, eta.default_scale(64), causal)
+        check_o(o, o_ref, "large scores")
+        check_lse(lse, lse_ref, "large scores lse")
+
+
+def _sampled_rows(N):
+    rows = {0, 1, 127, 128, 129, 255, 256, N // 2, N - 129, N - 128, N - 2, N - 1}
+    rng = np.random.default_rng(0)
+    rows |= set(int(r) for r in rng.integers(0, N, 20))
+    return sorted(r for r in rows if 0 <= r < N)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_prefill_d64_full_config_sampled(causal):
+    """Prefill MHA B=1, H=32, N=4096, d=64 in the benchmark's launch configuration; sampled rows of every
+    head compared with the oracle."""
+    B, H, N, d = 1, 32, 4096, 64
+    q, k, v = inputs.dense_qkv(inputs.PREFILL_D64, B, H, N, d, device=DEV)
+    scale = eta.default_scale(d)
+    o, lse = eta.attn_fwd(q, k, v, causal=causal, scale=scale)
+    assert eta.status() == 0
+    rows = _sampled_rows(N)
+    o_ref, lse_ref = oracle.attn(q, k, v, scale, causal, rows=rows)
+    check_o(o[:, :, rows], o_ref, "C2 sampled")
+    check_lse(lse[:, :, rows], lse_ref, "C2 lse")
+
+
+def test_prefill_d128_full_config_sampled():
+    """Prefill MHA B=8, H=32, N=4096, d=128, causal; sampled rows of sampled (batch, head) pairs."""
+    B, H, N, d = 8, 32, 4096, 128
+    q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, B, H, N, d, device=DEV)
+    scale = eta.default_scale(d)
+    o, lse = eta.attn_fwd(q, k, v, causal=True, scale=scale)
+    assert eta.status() == 0
+    rows = _sampled_rows(N)
+    for b, h in ((0, 0), (3, 17), (7, 31)):
+        sl = lambda x: x[b:b + 1, h:h + 1]
+        o_ref, lse_ref = oracle.attn(sl(q), sl(k), sl(v), scale, True, rows=rows)
+        check_o(sl(o)[:, :, rows], o_ref, f"C3 b={b} h={h}")
+        check_lse(sl(lse)[:, :, rows], lse_ref, "C3 lse")
+
+
+@pytest.mark.parametrize("N", [1024, 8192, 32768])
+def test_prefill_d128_sweep_sampled(N):
+    """N sweep at B=1, H=32, d=128, causal: sampled rows of three heads."""
+    q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, 1, 32, N, 128, device=DEV)
+    scale = eta.default_scale(128)
+    o, lse = eta.attn_fwd(q, k, v, causal=True, scale=scale)
+    assert eta.status() == 0
+    rows = _sampled_rows(N)[:24]
+    for h in (0, 13, 31):
+        sl = lambda x: x[:, h:h + 1]
+        o_ref, lse_ref = oracle.attn(sl(q), sl(k), sl(v), scale, True, rows=rows)
+        check_o(sl(o)[:, :, rows], o_ref, f"sweep N={N} h={h}")
+        check_lse(sl(lse)[:, :, rows], lse_ref, "sweep lse")

@@ -1,0 +1,72 @@
+"""attn_fwd_varlen and hstu_fwd_jagged (packed sequences) against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import exact_tiled_attention_43_b200 as eta
+import oracle
+from exact_tiled_attention_43_b200 import inputs
+from parity import check_hstu, check_lse, check_o
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+EDGE_LENS = [1, 127, 128, 129, 0, 255, 256, 257, 300, 2]
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_edge_lengths(d, causal):
+    cu = inputs.cu_seqlens(EDGE_LENS)
+    T, H = int(cu[-1]), 3
+    q, k, v = (t.to(DEV) for t in inputs.jagged_qkv(11, T, H, d))
+    scale = eta.default_scale(d)
+    o, lse = eta.attn_fwd_varlen(q, k, v, cu.to(DEV), max(EDGE_LENS), causal=causal, scale=scale)
+    assert eta.status() == 0
+    o_ref, lse_ref = oracle.attn_varlen(q, k, v, cu, scale, causal)
+    check_o(o, o_ref, f"varlen d={d} causal={causal}")
+    check_lse(lse, lse_ref, "varlen lse")
+
+
+def test_varlen_equals_dense_for_one_sequence():
+    q, k, v = (t.to(DEV) for t in inputs.dense_qkv(12, 1, 4, 777, 64))
+    od, ld = eta.attn_fwd(q, k, v, causal=True)
+    pk = lambda x: x[0].transpose(0, 1).contiguous()
+    cu = torch.tensor([0, 777], dtype=torch.int32, device=DEV)
+    ov, lv = eta.attn_fwd_varlen(pk(q), pk(k), pk(v), cu, 777, causal=True)
+    assert torch.equal(ov, pk(od)) and torch.equal(lv, ld[0].t())
+
+
+def test_varlen_bad_cu_seqlens_sets_status():
+    q, k, v = (t.to(DEV) for t in inputs.jagged_qkv(13, 300, 1, 64))
+    cu = torch.tensor([0, 200, 100, 300], dtype=torch.int32, device=DEV)
+    eta.attn_fwd_varlen(q, k, v, cu, 300)
+    assert eta.status() == eta.ETA_DEV_BAD_CUSEQ
+    cu = torch.tensor([0, 300], dtype=torch.int32, device=DEV)
+    eta.attn_fwd_varlen(q, k, v, cu, 256)  # a sequence longer than max_len
+    assert eta.status() == eta.ETA_DEV_BAD_CUSEQ
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("inv_n", [1.0 / 4096, 1.0])
+def test_hstu_edge_lengths(d, inv_n):
+    cu = inputs.cu_seqlens(EDGE_LENS)
+    T, H = int(cu[-1]), 2
+    q, k, v = (t.to(DEV) for t in inputs.jagged_qkv(inputs.HSTU_JAGGED, T, H, d, std=0.5))
+    alpha = 1.0 / np.sqrt(d)
+    o = eta.hstu_fwd_jagged(q, k, v, cu.to(DEV), max(EDGE_LENS), alpha, inv_n)
+    assert eta.status() == 0
+    o_ref = oracle.hstu_jagged(q, k, v, cu, alpha, inv_n)
+    check_hstu(o, o_ref, f"hstu d={d} inv_n={inv_n}")
+
+
+def test_hstu_full_config():
+    """HSTU jagged: 16 sequences, H=4, d=64, lengths U[256, 4096], N(0, 0.5^2) inputs, alpha = 1/sqrt(d),
+    n = 4096 -- every output element compared."""
+    lens = inputs.uniform_lengths(inputs.HSTU_JAGGED, 16, 256, 4096)
+    cu = inputs.cu_seqlens(lens)
+    T = int(cu[-1])
+    q, k, v = inputs.jagged_qkv(inputs.HSTU_JAGGED, T, 4, 64, std=0.5, device=DEV)
+    o = eta.hstu_fwd_jagged(q, k, v, cu.to(DEV), 4096, 0.125, 1.0 / 4096)
+    assert eta.status() == 0
+    o_ref = oracle.hstu_jagged(q, k, v, cu, 0.125, 1.0 / 4096)
+    check_hstu(o, o_ref, "hstu C4")
