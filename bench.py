@@ -1,0 +1,486 @@
+"""Benchmark: exact tiled attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extra]
+
+A step is one pass of the hot path over the headline workload: prefill MHA with B=1, H=32, N=4096, d=64
+(bf16 Q/K/V iid N(0,1)), one non-causal and one causal forward (O bf16 + fp32 lse).  `value` is
+TFLOP/s with the 4 n^2 d convention (halved for causal) over the whole job; L2 is flushed (a 256 MiB
+write) before every timed step, outside the timed events.  The same JSON line carries the roofline of the
+prefill kernel, an end-to-end number through the public API with host buffers, the oracle timed on the
+host cores, the SM clocks seen during timing, and (unless --no-extra) the other workloads of the method:
+prefill d=128 (B=8, causal) and its N sweep, HSTU over jagged sequences, and the decode step (GB/s).
+
+--impl reference times the fp64 CPU oracle (the only reference implementation this method has) on the
+same workload and metric, each step a bounded sample of it.
+Multi-GPU: one process per GPU (torchrun); every rank runs the same workload on its own GPU (weak
+scaling, no data-path collective); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+HEADLINE = dict(B=1, H=32, N=4096, d=64)
+METRIC = "attn fwd TFLOP/s (4n²d) & % of B200 BF16 peak; decode HBM GB/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------------------------------------ utils
+def attn_flops(B, H, N, d, causal):
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def hstu_flops(lengths, H, d):
+    return sum(2.0 * H * int(L) * int(L) * d for L in lengths)
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("ptx.cuh", "prefill.cuh", "decode.cuh"):
+        with open(os.path.join(ROOT, "exact_tiled_attention_43_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_tag):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 3 and parts[0] == kernel_tag and parts[1] == want:
+            return float(parts[2])
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    BAD = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40, "sw_power_cap": 0x4,
+           "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.BAD.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def timed_steps(step_fn, steps, warmup, flush_buf, stream, dist_ctx):
+    """W untimed warm-up steps; then K steps, each preceded by an L2 flush outside its CUDA events.
+    Returns (total ms of the K steps on the device, per-step ms list)."""
+    for _ in range(warmup):
+        step_fn()
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            flush_buf.fill_(1)
+            a.record(stream)
+            step_fn()
+            b.record(stream)
+    torch.cuda.synchronize()
+    dist_ctx.barrier()
+    torch.cuda.synchronize()
+    per = [a.elapsed_time(b) for a, b in evs]
+    return sum(per), per
+
+
+class DistCtx:
+    def __init__(self, n_gpus):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.on = self.world > 1
+        if self.on:
+            import datetime
+
+            import torch.distributed as dist
+
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+            self.dist = dist
+
+    def barrier(self):
+        if self.on:
+            self.dist.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.on:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.on:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------------------------------------ CPU
+def cpu_oracle_sample(budget_s=12.0):
+    """Times the fp64 oracle on a bounded sample of the headline workload (whole heads, non-causal +
+    causal), sized to about `budget_s` seconds.  Returns a cpu_baseline dict (TFLOP/s, 4 n^2 d convention)."""
+    import oracle
+    from exact_tiled_attention_43_b200 import inputs
+
+    B, H, N, d = HEADLINE["B"], HEADLINE["H"], HEADLINE["N"], HEADLINE["d"]
+    q, k, v = inputs.dense_qkv(inputs.PREFILL_D64, B, H, N, d)
+    scale = float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))
+    oracle.build()
+    # calibrate on one head
+    t0 = time.perf_counter()
+    for causal in (False, True):
+        oracle.attn(q[:, :1], k[:, :1], v[:, :1], scale, causal)
+    t1 = time.perf_counter() - t0
+    nh = int(max(1, min(H, budget_s // max(t1, 1e-3))))
+    t0 = time.perf_counter()
+    for causal in (False, True):
+        oracle.attn(q[:, :nh], k[:, :nh], v[:, :nh], scale, causal)
+    el = time.perf_counter() - t0
+    flops = attn_flops(B, nh, N, d, False) + attn_flops(B, nh, N, d, True)
+    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{nh} of {H} heads (B=1, N=4096, d=64), non-causal + causal, full rows, {el:.1f} s",
+            "seconds": el}
+
+
+def run_reference(args):
+    """The reference arm: the fp64 oracle on the host cores, same workload and metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from exact_tiled_attention_43_b200 import inputs
+
+    oracle.build()
+    B, H, N, d = HEADLINE["B"], HEADLINE["H"], HEADLINE["N"], HEADLINE["d"]
+    q, k, v = inputs.dense_qkv(inputs.PREFILL_D64, B, H, N, d)
+    scale = float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))
+    # each step: one head, non-causal + causal, rows sampled evenly (bounded CPU time per step)
+    rows = list(range(0, N, 32))
+    step_flops = sum(4.0 * (N if not c else (r + 1)) * d for c in (False, True) for r in rows)
+
+    def step():
+        for causal in (False, True):
+            oracle.attn(q[:, :1], k[:, :1], v[:, :1], scale, causal, rows=rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    val = step_flops * args.steps / el / 1e12
+    cores = oracle.num_threads()
+    sample = "per step: 1 of 32 heads, every 32nd query row (128 rows), non-causal + causal, N=4096, d=64"
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config(),
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config():
+    return {"workload": "prefill MHA B=1 H=32 N=4096 d=64 bf16, non-causal + causal per step",
+            "B": 1, "H": 32, "N": 4096, "d": 64, "o_dtype": "bf16", "lse": "fp32",
+            "scale": "1/sqrt(d)", "l2": "flushed before every timed step (256 MiB write), outside the events",
+            "parallelism": "replicas: each rank runs the whole workload on its own GPU"}
+
+
+# ------------------------------------------------------------------------------------------------ GPU
+def run_ours(args):
+    import exact_tiled_attention_43_b200 as eta
+    from exact_tiled_attention_43_b200 import inputs
+
+    ctx = DistCtx(args.gpus)
+    dev = torch.device("cuda", ctx.local)
+    torch.cuda.set_device(dev)
+    eta.lib()
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    B, H, N, d = HEADLINE["B"], HEADLINE["H"], HEADLINE["N"], HEADLINE["d"]
+    q, k, v = inputs.dense_qkv(inputs.PREFILL_D64, B, H, N, d, device=dev)
+    scale = eta.default_scale(d)
+    o_nc = torch.empty_like(q)
+    o_c = torch.empty_like(q)
+    l_nc = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    l_c = torch.empty_like(l_nc)
+    step_flops = attn_flops(B, H, N, d, False) + attn_flops(B, H, N, d, True)
+
+    # per-launch events for the roofline of the prefill kernel
+    launch_ms = []
+
+    def step():
+        eta.attn_fwd(q, k, v, causal=False, scale=scale, out=o_nc, lse=l_nc)
+        eta.attn_fwd(q, k, v, causal=True, scale=scale, out=o_c, lse=l_c)
+
+    with ClockSampler(ctx.local) as clk:
+        total_ms, per = timed_steps(step, args.steps, args.warmup, flush, stream, ctx)
+    clocks = clk.summary()
+    # per-launch durations (same kernel, two launches per step), measured in a second timed pass
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for _ in range(min(args.steps, 50)):
+        flush.fill_(1)
+        ev[0].record()
+        eta.attn_fwd(q, k, v, causal=False, scale=scale, out=o_nc, lse=l_nc)
+        ev[1].record()
+        eta.attn_fwd(q, k, v, causal=True, scale=scale, out=o_c, lse=l_c)
+        ev[2].record()
+        torch.cuda.synchronize()
+        launch_ms.append((ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2])))
+    assert eta.status() == 0
+
+    t_max = ctx.max(total_ms)
+    value = step_flops * args.steps * ctx.world / (t_max * 1e-3) / 1e12
+    nc_ms = statistics.mean(a for a, _ in launch_ms)
+    c_ms = statistics.mean(b for _, b in launch_ms)
+    achieved = (attn_flops(B, H, N, d, False) + attn_flops(B, H, N, d, True)) / ((nc_ms + c_ms) * 1e-3) / 1e12
+    traffic = recorded_traffic("prefill_d64")
+
+    # ---- end to end through the public API with pinned host buffers
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty(o_nc.shape, dtype=o_nc.dtype).pin_memory()
+    oh2 = torch.empty_like(oh).pin_memory()
+    lh = torch.empty(l_nc.shape, dtype=torch.float32).pin_memory()
+    lh2 = torch.empty_like(lh).pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        eta.attn_fwd(qd, kd, vd, causal=False, scale=scale, out=o_nc, lse=l_nc)
+        eta.attn_fwd(qd, kd, vd, causal=True, scale=scale, out=o_c, lse=l_c)
+        oh.copy_(o_nc, non_blocking=True)
+        lh.copy_(l_nc, non_blocking=True)
+        oh2.copy_(o_c, non_blocking=True)
+        lh2.copy_(l_c, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 50))
+    e2e_ms, _ = timed_steps(e2e_step, e2e_steps, args.warmup, flush, stream, ctx)
+    e2e_ms = ctx.max(e2e_ms)
+    h2d = 3 * q.numel() * 2
+    d2h = 2 * (o_nc.numel() * 2 + l_nc.numel() * 4)
+
+    extra = {} if args.no_extra else run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks)
+
+    line = None
+    if ctx.rank == 0:
+        cpu = None
+        if ctx.world == 1 and not args.no_cpu:
+            cpu = cpu_oracle_sample()
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ctx.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_max / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (iid N(0,1) bf16, fixed seeds)",
+            "config": _config(),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                         "kernel": "prefill_kernel<64, dense>",
+                         "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)",
+                         "launch_ms": {"noncausal": nc_ms, "causal": c_ms}},
+            "cpu_baseline": cpu,
+            "e2e": {"value": step_flops * e2e_steps * ctx.world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+            "extra": extra,
+        }
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    return line
+
+
+def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
+    """The method's other workloads, each timed the same way (few steps)."""
+    out = {}
+    K, W = max(3, min(args.steps, 20)), max(3, args.warmup)
+    pk = peaks["bf16_tflops"]
+
+    # prefill d=128, B=8, causal
+    q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, 8, 32, 4096, 128, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    ms, _ = timed_steps(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse), K, W, flush, stream, ctx)
+    f = attn_flops(8, 32, 4096, 128, True)
+    tf = f * K / (ctx.max(ms) * 1e-3) / 1e12
+    out["prefill_B8_H32_N4096_d128_causal"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+                                               "frac_of_peak": tf / pk}
+    del q, k, v, o, lse
+    for N in (1024, 8192, 32768):
+        q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, 1, 32, N, 128, device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        ms, _ = timed_steps(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse), K, W, flush, stream, ctx)
+        tf = attn_flops(1, 32, N, 128, True) * K / (ctx.max(ms) * 1e-3) / 1e12
+        out[f"prefill_B1_H32_N{N}_d128_causal"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+                                                   "frac_of_peak": tf / pk}
+        del q, k, v, o, lse
+
+    # HSTU jagged: 16 sequences, H=4, d=64, lengths U[256, 4096]
+    lens = inputs.uniform_lengths(inputs.HSTU_JAGGED, 16, 256, 4096)
+    cu = inputs.cu_seqlens(lens).to(dev)
+    T = int(lens.sum())
+    q, k, v = inputs.jagged_qkv(inputs.HSTU_JAGGED, T, 4, 64, std=0.5, device=dev)
+    o = torch.empty_like(q)
+    ms, _ = timed_steps(lambda: eta.hstu_fwd_jagged(q, k, v, cu, 4096, 0.125, 1.0 / 4096, out=o), K, W, flush,
+                        stream, ctx)
+    tf = hstu_flops(lens.tolist(), 4, 64) * K / (ctx.max(ms) * 1e-3) / 1e12
+    out["hstu_jagged_S16_H4_d64"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K, "frac_of_peak": tf / pk,
+                                     "T": T}
+    del q, k, v, o
+
+    # decode: batch 64, H=32, d=128, lengths U[8192, 32768] (inputs far larger than L2: no flush needed)
+    B, H, d, Lmax = 64, 32, 128, 32768
+    lens = inputs.uniform_lengths(inputs.DECODE, B, 8192, 32768)
+    q, kc, vc, kl = inputs.decode_inputs(inputs.DECODE, B, H, Lmax, d, lens, device=dev)
+    kl = kl.to(dev)
+    ws = torch.empty(eta.attn_decode_workspace_size(B, H, Lmax, d), dtype=torch.uint8, device=dev)
+    od = torch.empty((B, H, d), dtype=torch.bfloat16, device=dev)
+    ld = torch.empty((B, H), dtype=torch.float32, device=dev)
+    ms, _ = timed_steps(lambda: eta.attn_decode(q, kc, vc, kl, workspace=ws, out=od, lse=ld), K, W, flush, stream,
+                        ctx)
+    nbytes = 2.0 * H * d * 2 * float(lens.sum()) + q.numel() * 2 + od.numel() * 2 + ld.numel() * 4
+    gbs = nbytes * K / (ctx.max(ms) * 1e-3) / 1e9
+    out["decode_B64_H32_d128_L8k-32k"] = {"value": gbs, "unit": "GB/s", "ms_per_step": ms / K,
+                                          "frac_of_peak": gbs / peaks["hbm_gbs"], "bytes_per_step": nbytes}
+    del q, kc, vc, ws
+    torch.cuda.empty_cache()
+    assert eta.status() == 0
+    return out
+
+
+CASES = {
+    # name: (kind, shape) -- small named cases for profiler captures (no JSON line, just launches)
+    "prefill_d64_headline": ("dense", dict(B=1, H=32, N=4096, d=64)),
+    "prefill_d64_b4": ("dense", dict(B=4, H=32, N=4096, d=64)),
+    "prefill_d128_b2": ("dense", dict(B=2, H=32, N=4096, d=128)),
+    "hstu_jagged": ("hstu", dict(S=16, H=4, d=64)),
+    "decode_b2": ("decode", dict(B=2, H=32, d=128, Lmax=32768)),
+}
+
+
+def run_case(args):
+    """Runs one named case `--warmup` + `--steps` times (both causal modes for dense prefill); used as the
+    target of ncu captures."""
+    import exact_tiled_attention_43_b200 as eta
+    from exact_tiled_attention_43_b200 import inputs
+
+    kind, s = CASES[args.case]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if kind == "dense":
+        q, k, v = inputs.dense_qkv(inputs.PREFILL_D64 if s["d"] == 64 else inputs.PREFILL_D128, s["B"], s["H"],
+                                   s["N"], s["d"], device=dev)
+        fns = [lambda: eta.attn_fwd(q, k, v, causal=False), lambda: eta.attn_fwd(q, k, v, causal=True)]
+    elif kind == "hstu":
+        lens = inputs.uniform_lengths(inputs.HSTU_JAGGED, s["S"], 256, 4096)
+        cu = inputs.cu_seqlens(lens).to(dev)
+        q, k, v = inputs.jagged_qkv(inputs.HSTU_JAGGED, int(lens.sum()), s["H"], s["d"], std=0.5, device=dev)
+        fns = [lambda: eta.hstu_fwd_jagged(q, k, v, cu, 4096, 0.125, 1.0 / 4096)]
+    else:
+        lens = inputs.uniform_lengths(inputs.DECODE, 64, 8192, 32768)[: s["B"]]
+        q, kc, vc, kl = inputs.decode_inputs(inputs.DECODE, s["B"], s["H"], s["Lmax"], s["d"], lens, device=dev)
+        kl = kl.to(dev)
+        fns = [lambda: eta.attn_decode(q, kc, vc, kl)]
+    for _ in range(args.warmup + args.steps):
+        for f in fns:
+            f()
+    torch.cuda.synchronize()
+    assert eta.status() == 0
+    print(f"case {args.case}: ok", flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--case", choices=sorted(CASES), help="run one small named case (profiling target)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.case:
+        run_case(args)
+    elif args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
