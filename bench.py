@@ -153,18 +153,24 @@ def timed_steps(step_fn, steps, warmup, flush_buf, stream, dist_ctx):
 
 
 class DistCtx:
-    def __init__(self, n_gpus):
+    """One process per GPU: rank/world from the torchrun environment; the process group is used only for
+    barriers and the max-over-ranks of the device time (no data-path collective: every rank runs the whole
+    workload on its own GPU).  `backend="gloo"` runs the same logic on CPU (tests)."""
+
+    def __init__(self, backend="nccl"):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.on = self.world > 1
+        self.device = "cuda" if backend == "nccl" else "cpu"
         if self.on:
             import datetime
 
             import torch.distributed as dist
 
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
             self.dist = dist
 
     def barrier(self):
@@ -174,7 +180,7 @@ class DistCtx:
     def max(self, x: float) -> float:
         if not self.on:
             return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
         self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
         return float(t.item())
 
@@ -182,6 +188,11 @@ class DistCtx:
         if self.on:
             self.dist.barrier()
             self.dist.destroy_process_group()
+
+
+def job_throughput(units_per_step: float, steps: int, world: int, t_max_ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed divided by the slowest rank's device time."""
+    return units_per_step * steps * world / (t_max_ms * 1e-3)
 
 
 # ------------------------------------------------------------------------------------------------ CPU
@@ -261,7 +272,7 @@ def run_ours(args):
     import exact_tiled_attention_43_b200 as eta
     from exact_tiled_attention_43_b200 import inputs
 
-    ctx = DistCtx(args.gpus)
+    ctx = DistCtx("nccl")
     dev = torch.device("cuda", ctx.local)
     torch.cuda.set_device(dev)
     eta.lib()
@@ -302,7 +313,7 @@ def run_ours(args):
     assert eta.status() == 0
 
     t_max = ctx.max(total_ms)
-    value = step_flops * args.steps * ctx.world / (t_max * 1e-3) / 1e12
+    value = job_throughput(step_flops, args.steps, ctx.world, t_max) / 1e12
     nc_ms = statistics.mean(a for a, _ in launch_ms)
     c_ms = statistics.mean(b for _, b in launch_ms)
     achieved = (attn_flops(B, H, N, d, False) + attn_flops(B, H, N, d, True)) / ((nc_ms + c_ms) * 1e-3) / 1e12
