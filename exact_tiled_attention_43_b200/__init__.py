@@ -33,6 +33,7 @@ SIGNATURES = {
     "hstu_fwd_jagged": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _F, _VP]),
     "attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "attn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _SZ, _VP]),
+    "attn_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP]),
     "eta_status": (_I, [_VP]),
     "eta_strerror": (ctypes.c_char_p, [_I]),
     "eta_set_wait_timeout_ns": (None, [_LL]),
@@ -190,6 +191,32 @@ def attn_decode(q, kcache, vcache, kv_lens, scale: float | None = None, workspac
     rc = lib().attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kv_lens), _ptr(out), _ptr(lse), B, H, Lmax, d,
                            scale, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     _check(rc, "attn_decode")
+    return out, lse
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES
+
+
+def attn_decode_noalloc(q, kcache, vcache, kv_lens, scale: float | None = None, out=None, lse=None, stream=None):
+    """attn_decode without a workspace: the library's fixed device scratch (NOALLOC_SCRATCH_BYTES) holds the
+    split partials, for callers that cannot allocate device memory at call time.  Calls whose GPU work
+    overlaps race on that shared scratch; the first call on a device should precede any stream capture."""
+    torch = _torch()
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kcache, "kcache", torch.bfloat16, 4)
+    _need(vcache, "vcache", torch.bfloat16, 4)
+    _need(kv_lens, "kv_lens", torch.int32, 1)
+    B, H, Lmax, d = kcache.shape
+    if vcache.shape != kcache.shape or q.shape != (B, H, d) or kv_lens.shape != (B,):
+        raise ValueError("inconsistent decode shapes")
+    if out is None:
+        out = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    scale = default_scale(d) if scale is None else float(scale)
+    rc = lib().attn_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kv_lens), _ptr(out), _ptr(lse), B, H,
+                                   Lmax, d, scale, _stream_ptr(stream))
+    _check(rc, "attn_decode_noalloc")
     return out, lse
 
 

@@ -290,3 +290,54 @@ int eta_selftest_wait_timeout(void *stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// Allocation-free decode: the split-KV partials live in a fixed file-scope device array instead of a
+// caller-provided workspace.  Same kernels as attn_decode.
+// ------------------------------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ETA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch per device ordinal, looked up once with that device current.  In
+// host code the array's name is only a host-side stand-in; kernels must be given this address.
+void *noalloc_scratch_ptr(int *rc) {
+  static void *ptrs[64];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *rc = ETA_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      *rc = ETA_ERR_CUDA;
+      return nullptr;
+    }
+    ptrs[dev] = p;
+  }
+  *rc = ETA_OK;
+  return ptrs[dev];
+}
+
+}  // namespace
+
+extern "C" int attn_decode_noalloc(const void *q, const void *kcache, const void *vcache, const int *kv_lens,
+                                   void *o, float *lse, int B, int H, int Lmax, int d, float scale, void *stream) {
+  if (B > 0 && H > 0 && Lmax > 0 && (d == 64 || d == 128) &&
+      decode_ws_bytes(B, H, Lmax, d) > (size_t)ETA_NOALLOC_SCRATCH_BYTES)
+    return ETA_ERR_WORKSPACE;
+  // Argument checks that need no device come first (same order as attn_decode).
+  if (!q || !kcache || !vcache || !kv_lens || !o) return ETA_ERR_NULL;
+  if (d != 64 && d != 128) return ETA_ERR_HEAD_DIM;
+  if (B <= 0 || H <= 0 || Lmax <= 0) return ETA_ERR_SHAPE;
+  int rc = check_device();
+  if (rc != ETA_OK) return rc;
+  void *scratch = noalloc_scratch_ptr(&rc);
+  if (rc != ETA_OK) return rc;
+  return attn_decode(q, kcache, vcache, kv_lens, o, lse, B, H, Lmax, d, scale, scratch,
+                     (size_t)ETA_NOALLOC_SCRATCH_BYTES, stream);
+}
+

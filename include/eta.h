@@ -135,6 +135,28 @@ ETA_API int attn_decode(const void *q, const void *kcache, const void *vcache, c
                 void *stream);
 
 /*
+ * attn_decode_noalloc -- the same decode step as attn_decode, for callers that cannot allocate device memory
+ * when they call: for example a plugin running inside a host engine that owns all device memory and forbids
+ * allocation in its enqueue step, or a latency-critical loop that cannot afford cudaMalloc's implicit
+ * device synchronisation.  It takes no workspace argument: the split-KV partial results go to a fixed
+ * scratch array of ETA_NOALLOC_SCRATCH_BYTES that the library holds in device memory (one copy on every GPU
+ * that loads the library, kept until the process exits).  The paper has no counterpart; it is an
+ * interface convenience around the decode kernels.
+ *   Arguments, layouts and results are exactly those of attn_decode (minus workspace / workspace_bytes).
+ *   The first call on a device, with that device current, looks up the scratch array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.  No call allocates or frees
+ *   memory.
+ *   Returns ETA_ERR_WORKSPACE, and enqueues nothing, when attn_decode_workspace_size(B, H, Lmax, d) exceeds
+ *   ETA_NOALLOC_SCRATCH_BYTES; other errors as attn_decode.
+ *   All calls on a device share the one scratch array, which keeps the last call's contents (every value a
+ *   call reads is written earlier by that same call, so nothing needs clearing).  Calls whose GPU work
+ *   overlaps -- on different streams, or from different host threads -- race on it: serialise them.
+ */
+#define ETA_NOALLOC_SCRATCH_BYTES (8u << 20)
+ETA_API int attn_decode_noalloc(const void *q, const void *kcache, const void *vcache, const int *kv_lens, void *o,
+                                float *lse, int B, int H, int Lmax, int d, float scale, void *stream);
+
+/*
  * eta_status -- synchronises `stream`, returns the device status word of the current device
  * (ETA_DEV_*; the first condition recorded since the last call) and clears it.  Returns ETA_ERR_CUDA if
  * the synchronisation or the copy failed.
