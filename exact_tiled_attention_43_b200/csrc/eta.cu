@@ -93,6 +93,7 @@ int launch_prefill(const void *q, const void *k, const void *v, bool packed, lon
   constexpr int smem = eta::PfCfg<D>::SMEM_BYTES;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ETA_ERR_CUDA;
+
   kern<<<grid, eta::PF_THREADS, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
 }
@@ -127,7 +128,7 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
     if (T_total == 0) return ETA_OK;  // nothing to compute
     const long long nblk = ((long long)max_len + 255) / 256;
     if (nblk > 65535) return ETA_ERR_SHAPE;
-    grid = dim3((unsigned)H, (unsigned)nblk, (unsigned)S);
+    grid = dim3((unsigned)H, (unsigned)S, (unsigned)nblk);
     n1 = H;
     n2 = T_total;
     p.max_len = max_len;
