@@ -93,7 +93,10 @@ int launch_prefill(const void *q, const void *k, const void *v, bool packed, lon
   constexpr int smem = eta::PfCfg<D>::SMEM_BYTES;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ETA_ERR_CUDA;
-
+  // The kernel re-splits its registers between warpgroups (setmaxnreg); the split only adds up when the
+  // build uses exactly PF_LAUNCH_REGS registers per thread, so refuse any other build.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != eta::PF_LAUNCH_REGS) return ETA_ERR_CUDA;
   kern<<<grid, eta::PF_THREADS, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
 }

@@ -43,7 +43,13 @@ namespace eta {
 constexpr int PF_BM = 128;            // query rows per Q tile (= TMEM lanes)
 constexpr int PF_BN = 128;            // keys per K/V tile
 constexpr int PF_SM_WARPS = 8;        // softmax warps: 2 Q tiles x 4 lane quarters (one thread per query row)
-constexpr int PF_THREADS = 32 * (3 + PF_SM_WARPS);  // + TMA warp + 2 MMA-issuer warps
+constexpr int PF_THREADS = 32 * (4 + PF_SM_WARPS);  // + control warpgroup: TMA, 2 MMA issuers, 1 spare
+// Register split (setmaxnreg): the CTA launches with PF_LAUNCH_REGS per thread; the control warpgroup drops
+// to PF_CTRL_REGS and the two softmax warpgroups grow to PF_SM_REGS.  The shares add up to the launch total
+// exactly, and the host refuses to launch a build whose register count is not PF_LAUNCH_REGS (a larger
+// request than the launch total would stall forever).
+constexpr int PF_LAUNCH_REGS = 168, PF_CTRL_REGS = 56, PF_SM_REGS = 224;
+static_assert(128 * PF_CTRL_REGS + 32 * PF_SM_WARPS * PF_SM_REGS == PF_THREADS * PF_LAUNCH_REGS, "register split");
 constexpr float PF_RESCALE_THRESHOLD = 8.0f;  // log2 units
 
 enum PrefillMode { MODE_DENSE = 0, MODE_VARLEN = 1, MODE_HSTU = 2 };
@@ -71,7 +77,9 @@ struct PfCfg {
   static constexpr int CHUNK_BYTES = PF_BM * 128;        // 128 rows x 128 B
   static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // one 128 x D bf16 tile
   static constexpr int NST = (D == 64) ? 8 : 4;          // K/V ring depth (each stage holds one tile)
-  static constexpr int POLY_PAIRS = 0;                    // of every 8 exp2 pairs, how many use the FMA pipe
+  // Of every 8 exp2 pairs, how many use the FMA-pipe polynomial instead of the MUFU.  Off: measured inside
+  // this kernel it costs more (issue slots, dependency chains) than the MUFU time it saves.
+  static constexpr int POLY_PAIRS = 0;
   // barriers: full/empty per stage, q, per tile {s_full, s_free, p_full, pv_done, mma_done}
   static constexpr int NBAR = 2 * NST + 1 + 2 * 5;
   static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + (2 + NST) * TILE_BYTES + NBAR * 8 + 16;
@@ -79,7 +87,8 @@ struct PfCfg {
   static constexpr uint32_t TM_P = 384;                  // P_t at TM_P + 64*t (D = 64); S_t's columns [0,64) (D = 128)
 };
 
-// Control warps: warp 0 streams Q, K, V with TMA; warps 1 and 2 issue the MMAs of Q tiles 0 and 1.
+// Control warpgroup: warp 0 streams Q, K, V with TMA; warps 1 and 2 issue the MMAs of Q tiles 0 and 1;
+// warp 3 has no role.
 template <int D, int MODE>
 __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CUtensorMap &tmK,
                                                 const CUtensorMap &tmV, const PrefillParams &p, uint8_t *smem,
@@ -230,7 +239,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
   }
 }
 
-// Softmax (or HSTU pointwise) warpgroups: warps 3-6 for Q tile 0, warps 7-10 for Q tile 1.  Thread
+// Softmax (or HSTU pointwise) warpgroups: warps 4-7 for Q tile 0, warps 8-11 for Q tile 1.  Thread
 // (quarter, lane) owns query row 32 quarter + lane of its tile (= its TMEM lane): it loads the S row from
 // TMEM, applies the mask, updates the running max and exp-sum, writes P (bf16) to TMEM, rescales its O row
 // when the max moved, and finally normalises O and stores O and lse.
@@ -256,7 +265,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   (void)sQ; (void)sKV; (void)full; (void)empty; (void)q_full; (void)s_full; (void)s_free;
   (void)p_full; (void)pv_done; (void)mma_done; (void)abort_flag; (void)HSTU; (void)PACKED;
-  const int t = (warp - 3) >> 2;
+  const int t = (warp - 4) >> 2;
   const int quarter = warp & 3;
   const int row = quarter * 32 + lane;
   const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
@@ -516,7 +525,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   // Each role runs to its own end; the teardown barrier (id 1, every thread of the CTA) is reached from
   // both sides.
-  if (warp < 3) {
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(PF_CTRL_REGS));
     prefill_control<D, MODE>(tmQ, tmK, tmV, p, smem, tmem, warp, lane, r0, h, bh, seq_start, n_t, n_kv);
     tc_fence_before();
     asm volatile("bar.sync 1, %0;" ::"n"(PF_THREADS) : "memory");
@@ -525,6 +535,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       tmem_dealloc(tmem, 512);
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(PF_SM_REGS));
     prefill_softmax<D, MODE>(p, smem, tmem, warp, lane, r0, L, h, bh, seq_start, causal, n_t);
     tc_fence_before();
     asm volatile("bar.sync 1, %0;" ::"n"(PF_THREADS) : "memory");
