@@ -36,6 +36,8 @@
 // consistently, so the result is exact (up to rounding) while most key tiles skip the O rescale.
 #pragma once
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace eta {
@@ -154,7 +156,79 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
           mbar_wait(&full[i % C::NST], (i / C::NST) & 1, nullptr, p.wait_ns);
       }
     }
-  } else if (warp == 1 || warp == 2) {
+  } else if (C::ALIAS_P && warp == 1) {
+    // ================================================================ single MMA issuer (P aliased into S)
+    // One thread issues both tiles' MMAs in the order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  tcgen05.mma
+    // operations issued by one thread execute in issue order, so S_t(j+1) -- which overwrites the columns
+    // holding P_t(j) -- needs no wait for PV_t(j) to complete; its commit also tracks that PV, so a softmax
+    // that has seen S_t(j+1) may rescale O_t.  The single ordered stream keeps the two softmax warpgroups
+    // half a period apart.
+    if (lane == 0) {
+      constexpr uint32_t ID_QK = idesc_bf16_f32(PF_BM, PF_BN, false);
+      constexpr uint32_t ID_PV = idesc_bf16_f32(PF_BM, D, true);
+      const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
+      auto issue_s = [&](int t, int st) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * C::CHUNK_BYTES + (uint32_t)(kk & 3) * 32u;
+          mma_ss(tmem + 128u * t, sdesc_sw128(sQa + t * C::TILE_BYTES + off, 16, 1024),
+                 sdesc_sw128(sKVa + st * C::TILE_BYTES + off, 16, 1024), ID_QK, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int st, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < PF_BN / 16; ++kk)
+          mma_ts(tmem + C::TM_O + (uint32_t)(D * t), tmem + 128u * t + 8u * kk,
+                 sdesc_sw128(sKVa + st * C::TILE_BYTES + kk * 2048, C::CHUNK_BYTES, 1024), ID_PV,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag, p.wait_ns);
+      if (ok && n_kv > 0) {
+        ok = mbar_wait(&full[0], 0, abort_flag, p.wait_ns);
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if (n_t[t] > 0) {
+              issue_s(t, 0);
+              mma_commit(&s_full[t]);
+            }
+          mma_commit(&empty[0]);
+        }
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int iv = 2 * j + 1, sv = iv % C::NST;
+        const int ik = 2 * j + 2, sk = ik % C::NST;
+        ok = mbar_wait(&full[sv], (iv / C::NST) & 1, abort_flag, p.wait_ns);
+        if (!ok) break;
+        bool k_ready = false;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || j >= n_t[t]) continue;
+          ok = mbar_wait(&p_full[t], j & 1, abort_flag, p.wait_ns);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(t, sv, j > 0);
+          mma_commit(&pv_done[t]);
+          if (j + 1 < n_t[t]) {
+            if (!k_ready) {
+              ok = mbar_wait(&full[sk], (ik / C::NST) & 1, abort_flag, p.wait_ns);
+              if (!ok) break;
+              k_ready = true;
+            }
+            issue_s(t, sk);
+            mma_commit(&s_full[t]);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&empty[sv]);
+        if (k_ready) mma_commit(&empty[sk]);
+      }
+      mma_commit(&mma_done[0]);
+      mbar_wait(&mma_done[0], 0, nullptr, p.wait_ns);
+    }
+    __syncwarp();
+  } else if (!C::ALIAS_P && (warp == 1 || warp == 2)) {
     // ================================================================ MMA issuer for Q tile t
     const int t = warp - 1;
     if (lane == 0) {
@@ -324,21 +398,26 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
       uint64_t rs_a = f2pack(0.f, 0.f), rs_b = f2pack(0.f, 0.f);
       // p = 2^(s * scale_log2 - m): pairs with (i % 8) < POLY_PAIRS go to the FMA-pipe polynomial on
       // unmasked tiles, the rest (and every element of a masked tile) to the MUFU.
+      auto exp_row = [&](auto use_poly) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const uint64_t x2 = fma_x2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), cs2, nm2);
-        float x0, x1, p0, p1;
-        f2unpack(x2, x0, x1);
-        if (!need_mask && (i % 8) < C::POLY_PAIRS) {
-          exp2_poly_x2(x0, x1, p0, p1);
-        } else {
-          p0 = ex2_approx(x0);
-          p1 = ex2_approx(x1);
+        for (int i = 0; i < 64; ++i) {
+          const uint64_t x2 =
+              fma_x2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), cs2, nm2);
+          float x0, x1, p0, p1;
+          f2unpack(x2, x0, x1);
+          if (decltype(use_poly)::value && (i % 8) < C::POLY_PAIRS) {
+            exp2_poly_x2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          if (i & 1) rs_b = add_x2(rs_b, f2pack(p0, p1));
+          else rs_a = add_x2(rs_a, f2pack(p0, p1));
+          pk[i] = pack_bf16x2(p0, p1);
         }
-        if (i & 1) rs_b = add_x2(rs_b, f2pack(p0, p1));
-        else rs_a = add_x2(rs_a, f2pack(p0, p1));
-        pk[i] = pack_bf16x2(p0, p1);
-      }
+      };
+      if (need_mask) exp_row(std::false_type{});
+      else exp_row(std::true_type{});
       float r0a, r1a, r2a, r3a;
       f2unpack(rs_a, r0a, r1a);
       f2unpack(rs_b, r2a, r3a);
@@ -502,7 +581,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 2);
+      mbar_init(&empty[i], C::ALIAS_P ? 1 : 2);  // released by each MMA issuer
     }
     mbar_init(q_full, 1);
     for (int t = 0; t < 2; ++t) {
