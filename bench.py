@@ -412,6 +412,19 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
                                      "T": T}
     del q, k, v, o
 
+    # HSTU at the HSTU page's own shape (QKV = 16, 4, 4096, 64: every sequence 4096 long) and at N = 8192
+    for S_, N_ in ((16, 4096), (16, 8192)):
+        lens = torch.full((S_,), N_, dtype=torch.int32)
+        cu = inputs.cu_seqlens(lens).to(dev)
+        q, k, v = inputs.jagged_qkv(inputs.HSTU_JAGGED, S_ * N_, 4, 64, std=0.5, device=dev)
+        o = torch.empty_like(q)
+        ms, _ = timed_steps(lambda: eta.hstu_fwd_jagged(q, k, v, cu, N_, 0.125, 1.0 / N_, out=o), K, W, flush,
+                            stream, ctx)
+        tf = hstu_flops(lens.tolist(), 4, 64) * K / (ctx.max(ms) * 1e-3) / 1e12
+        out[f"hstu_dense_S{S_}_H4_N{N_}_d64"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+                                                  "frac_of_peak": tf / pk}
+        del q, k, v, o
+
     # decode: batch 64, H=32, d=128, lengths U[8192, 32768] (inputs far larger than L2: no flush needed)
     B, H, d, Lmax = 64, 32, 128, 32768
     lens = inputs.uniform_lengths(inputs.DECODE, B, 8192, 32768)

@@ -10,10 +10,10 @@
 //  * one producer thread streams the split's K and V rows with 1-D bulk copies (cp.async.bulk, no
 //    multicast) into a DEC_STAGES-deep shared-memory ring of DEC_ROWS-row stages; each stage's K and V
 //    rows are contiguous in HBM because the cache is [B, H, Lmax, d].
-//  * four consumer warps take 8 rows of each stage; lane l holds d/32 consecutive elements of q, k and v,
+//  * eight consumer warps take 4 rows of each stage; lane l holds d/32 consecutive elements of q, k and v,
 //    so a row's dot product is d/32 FMAs per lane plus a 5-step xor-shuffle reduction.  Each warp keeps
 //    its own online-softmax state (running max m in log2 units, exp-sum l, fp32 output accumulator).
-//  * the four warp states are merged in shared memory, normalised, and written as one partial (o, lse).
+//  * the warp states are merged in shared memory, normalised, and written as one partial (o, lse).
 //  * a second kernel merges the splits of each (b, h) with logsumexp weights (exact) and writes o, lse.
 #pragma once
 
@@ -23,7 +23,7 @@ namespace eta {
 
 constexpr int DEC_ROWS = 32;          // cache rows per pipeline stage
 constexpr int DEC_STAGES = 4;         // pipeline depth
-constexpr int DEC_CWARPS = 4;         // consumer warps
+constexpr int DEC_CWARPS = 8;         // consumer warps (4 were compute-bound: 5.3 TB/s vs 7.3 with 8)
 constexpr int DEC_THREADS = 32 * (1 + DEC_CWARPS);
 
 // Rows per split: about Lmax/16, a multiple of the stage size, at most 1024 rows (512 KB of K+V at d=128).
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeP
 #pragma unroll
   for (int e = 0; e < EPL; ++e) wacc[cw][lane * EPL + e] = ok ? acc[e] : 0.f;
   asm volatile("bar.sync 1, %0;" ::"r"(32 * DEC_CWARPS) : "memory");
-  const int t = threadIdx.x - 32;  // 0 .. 127
+  const int t = threadIdx.x - 32;  // consumer thread index
   float M = -INFINITY;
 #pragma unroll
   for (int w = 0; w < DEC_CWARPS; ++w) M = fmaxf(M, wm[w]);

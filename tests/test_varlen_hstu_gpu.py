@@ -70,3 +70,21 @@ def test_hstu_full_config():
     assert eta.status() == 0
     o_ref = oracle.hstu_jagged(q, k, v, cu, 0.125, 1.0 / 4096)
     check_hstu(o, o_ref, "hstu C4")
+
+
+@pytest.mark.parametrize("N", [4096, 8192])
+def test_hstu_dense_page_shape_sampled(N):
+    """HSTU at the page's dense shape (16 sequences x 4 heads, every sequence N long, d = 64, n = N); the GPU
+    result of two sequences (first and last) and two heads is compared with the oracle run on them alone."""
+    S, H, d = 16, 4, 64
+    lens = [N] * S
+    cu = inputs.cu_seqlens(lens)
+    q, k, v = inputs.jagged_qkv(inputs.HSTU_JAGGED, S * N, H, d, std=0.5, device=DEV)
+    o = eta.hstu_fwd_jagged(q, k, v, cu.to(DEV), N, 0.125, 1.0 / N)
+    assert eta.status() == 0
+    for s in (0, S - 1):
+        a, b = s * N, (s + 1) * N
+        heads = [0, 3] if N == 4096 else [2]
+        sub = lambda x: x[a:b, heads].contiguous()
+        o_ref = oracle.hstu_jagged(sub(q), sub(k), sub(v), [0, N], 0.125, 1.0 / N)
+        check_hstu(sub(o), o_ref, f"hstu dense N={N} seq={s}")
