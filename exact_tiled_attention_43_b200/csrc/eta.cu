@@ -4,6 +4,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -34,6 +36,29 @@ int check_device() {
     cache[dev] = (major == 10 && minor == 0) ? 1 : -1;
   }
   return cache[dev] == 1 ? ETA_OK : ETA_ERR_DEVICE;
+}
+
+// Number of SMs of the current device (the persistent prefill grid), cached per device ordinal.
+int sm_count(int *out) {
+  static int cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ETA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return ETA_ERR_DEVICE;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      return ETA_ERR_CUDA;
+    cache[dev] = n;
+  }
+  *out = cache[dev];
+  return ETA_OK;
+}
+
+// Work-counter slot of the next prefill launch (round-robin over eta::PF_SCHED_SLOTS; a launch's last CTA
+// returns its slot to zero, so a slot is reusable once the launch that held it has finished).
+int next_sched_slot() {
+  static std::atomic<unsigned int> next{0};
+  return (int)(next.fetch_add(1u, std::memory_order_relaxed) % (unsigned int)eta::PF_SCHED_SLOTS);
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no -lcuda link).
@@ -115,27 +140,33 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   if (causal != 0 && causal != 1) return ETA_ERR_ARG;
   if (H <= 0 || H > 65535) return ETA_ERR_SHAPE;
   eta::PrefillParams p{};
-  dim3 grid;
-  long long n1, n2;
+  long long n1, n2, n_items;
   if (mode == eta::MODE_DENSE) {
     if (B <= 0 || N <= 0) return ETA_ERR_SHAPE;
     const long long bh = (long long)B * H;
     const long long nblk = ((long long)N + 255) / 256;
     if (bh > INT_MAX || nblk > 65535) return ETA_ERR_SHAPE;
-    grid = dim3((unsigned)bh, (unsigned)nblk, 1);
+    n_items = bh * nblk;
     n1 = N;
     n2 = bh;
     p.N = N;
+    p.BH = (int)bh;
+    p.nblk = (int)nblk;
   } else {
     if (S <= 0 || max_len <= 0 || T_total < 0 || S > 65535) return ETA_ERR_SHAPE;
     if (T_total == 0) return ETA_OK;  // nothing to compute
     const long long nblk = ((long long)max_len + 255) / 256;
     if (nblk > 65535) return ETA_ERR_SHAPE;
-    grid = dim3((unsigned)H, (unsigned)S, (unsigned)nblk);
+    n_items = (long long)S * H * nblk;
     n1 = H;
     n2 = T_total;
     p.max_len = max_len;
+    p.S = S;
+    p.nblk = (int)nblk;
   }
+  // The work counter may run past n_items by one per CTA: keep it far from 2^32.
+  if (n_items > (long long)INT_MAX) return ETA_ERR_SHAPE;
+  p.n_items = (int)n_items;
   if (mode == eta::MODE_HSTU) {
     if (!std::isfinite(alpha) || !finite_pos(inv_n)) return ETA_ERR_ARG;
     if (o_dtype != ETA_OUT_BF16) return ETA_ERR_ARG;
@@ -144,6 +175,10 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   }
   int rc = check_device();
   if (rc != ETA_OK) return rc;
+  int sms = 0;
+  if ((rc = sm_count(&sms)) != ETA_OK) return rc;
+  const dim3 grid((unsigned)std::min<long long>(n_items, sms), 1, 1);  // persistent: at most one CTA per SM
+  p.sched_slot = next_sched_slot();
   p.o = o;
   p.lse = (mode == eta::MODE_HSTU) ? nullptr : lse;
   p.cu_seqlens = cu_seqlens;

@@ -1,6 +1,6 @@
 // prefill.cuh -- fused exact attention forward (dense and packed/varlen) and HSTU pointwise attention, one
-// kernel template for B200 (sm_100a): TMA tile loads, tcgen05 MMAs accumulating in tensor memory (TMEM),
-// warp-specialised softmax, in-kernel causal mask with masked tiles skipped.
+// persistent kernel template for B200 (sm_100a): TMA tile loads, tcgen05 MMAs accumulating in tensor
+// memory (TMEM), warp-specialised softmax, in-kernel causal mask with masked tiles skipped.
 //
 // What it computes:
 //   softmax modes: O = softmax(scale * Q K^T [+ causal]) V and lse = ln sum_j exp(scale q_i.k_j), tile by
@@ -11,25 +11,29 @@
 //   HSTU mode: O = (silu(alpha Q K^T) * causal_mask * inv_n) V over packed sequences (the HSTU page,
 //     sections "先搞懂：HSTU到底难在哪？", "绝杀优化二：内置Mask生成", "绝杀优化三：Jagged变长张量").
 //
-// Work decomposition: one CTA owns 256 query rows of one (batch, head) -- two 128-row Q tiles -- and
-// streams the key/value tiles (128 rows each) its rows can see.  Causal tiles past the diagonal are never
-// loaded (the "after the diagonal: all zero, skip" class of the HSTU page's in-kernel mask); only the
-// diagonal tile and a ragged last tile evaluate a per-element mask.
+// Work decomposition: a work item is 256 query rows of one (batch, head) or (sequence, head) -- two 128-row
+// Q tiles -- streaming the key/value tiles (128 rows each) its rows can see.  Causal tiles past the
+// diagonal are never loaded (the "after the diagonal: all zero, skip" class of the HSTU page's in-kernel
+// mask); only the diagonal tile and a ragged last tile evaluate a per-element mask.  The grid is persistent
+// (at most one CTA per SM): CTAs take items heaviest-first from a device counter and keep their pipeline
+// running across items, so the next item's Q, K/V and first QK^T overlap the current item's epilogue.
 //
-// Roles (320 threads):
-//   warp 0      TMA producer: Q0,Q1 once, then K_0, V_0, K_1, V_1, ... through an NST-stage ring.
-//   warp 1      TMEM allocator + MMA issuer (one thread):  S_t = Q_t K_j^T (SS form) into TMEM,
-//               O_t += P_t V_j (TS form: P read from TMEM, V from shared memory).
-//   warps 2-5   softmax warpgroup for Q tile 0; warps 6-9 for Q tile 1.  Thread r of a group owns query
-//               row r = TMEM lane r: it loads its S row from TMEM, applies the mask, updates the running
-//               max/exp-sum, writes P (bf16) back into TMEM over the first 64 columns of S, rescales its
-//               O row when the max moved, and finally normalises O and stores O and lse.
-// The MMA thread interleaves the two tiles (PV_0, S_0', PV_1, S_1') so that one warpgroup's softmax runs
-// while the tensor core works for the other.
+// Roles (12 warps):
+//   warp 0      work fetcher + TMA producer: publishes each item to the other roles through a 2-deep ring,
+//               then loads its Q0, Q1 and K_0, V_0, K_1, V_1, ... through an NST-stage ring.
+//   warps 1, 2  MMA issuers (one thread each; warp 1 also owns TMEM):  S_t = Q_t K_j^T (SS form) into
+//               TMEM, O_t += P_t V_j (TS form: P read from TMEM, V from shared memory).
+//   warp 3      no role.
+//   warps 4-11  two softmax warpgroups, one per Q tile; thread r owns query row r = TMEM lane r.
 //
-// TMEM (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D);
-// P_t aliases the first 64 columns of S_t, so S_t of the next key tile is issued only after the MMA that
-// reads P_t has completed.
+// TMEM (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D).
+//   D = 64: P_t has its own columns [384+64t, 448+64t); issuer 1+t serves Q tile t and issues the next
+//           S_t as soon as the softmax has copied S_t to registers.
+//   D = 128: TMEM is full; P_t overwrites the first 64 columns of S_t and one issuer (warp 1) runs
+//           PV_0(j), S_0(j+1), PV_1(j), S_1(j+1) with no wait between a PV and the next QK^T: tcgen05.mma
+//           operations issued by one thread execute in issue order, so the QK^T's writes follow the PV's
+//           reads of P, and the QK^T's commit also covers the PV (a softmax that has seen the new S may
+//           rescale O).  The single ordered stream keeps the two softmax warpgroups half a period apart.
 //
 // Online-softmax rescale is conditional: the running max used for exponentiation is only raised when a
 // row's block max exceeds it by more than 8 (log2 units).  The final O / l and lse use the same stale max
@@ -37,10 +41,21 @@
 #pragma once
 
 #include <type_traits>
+#include <utility>
 
 #include "ptx.cuh"
 
 namespace eta {
+
+// Calls f(std::integral_constant<int, i>) for i = 0 .. N-1 (a loop whose index is a compile-time constant).
+template <int N, typename F, int... I>
+__device__ __forceinline__ void eta_static_for_impl(F &&f, std::integer_sequence<int, I...>) {
+  (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void eta_static_for(F &&f) {
+  eta_static_for_impl<N>(f, std::make_integer_sequence<int, N>{});
+}
 
 constexpr int PF_BM = 128;            // query rows per Q tile (= TMEM lanes)
 constexpr int PF_BN = 128;            // keys per K/V tile
@@ -53,6 +68,11 @@ constexpr int PF_THREADS = 32 * (4 + PF_SM_WARPS);  // + control warpgroup: TMA,
 constexpr int PF_LAUNCH_REGS = 168, PF_CTRL_REGS = 56, PF_SM_REGS = 224;
 static_assert(128 * PF_CTRL_REGS + 32 * PF_SM_WARPS * PF_SM_REGS == PF_THREADS * PF_LAUNCH_REGS, "register split");
 constexpr float PF_RESCALE_THRESHOLD = 8.0f;  // log2 units
+// Work counters of the persistent scheduler, one pair per launch in flight, handed out round-robin by the
+// host: [slot][0] = next item, [slot][1] = CTAs finished.  The last CTA of a launch resets its pair to zero
+// for the launch that reuses the slot.
+constexpr int PF_SCHED_SLOTS = 256;
+__device__ unsigned int g_pf_sched[PF_SCHED_SLOTS][2];
 
 enum PrefillMode { MODE_DENSE = 0, MODE_VARLEN = 1, MODE_HSTU = 2 };
 
@@ -61,6 +81,10 @@ struct PrefillParams {
   float *lse;              // dense: [B,H,N]; packed: [T,H]; may be null
   const int *cu_seqlens;   // packed modes: [S+1]
   int H, N, max_len;       // N: dense sequence length
+  int BH, S;               // dense: B*H; packed: number of sequences
+  int nblk;                // 256-row blocks per (batch|sequence, head)
+  int n_items;             // dense: nblk * BH; packed: nblk * S * H
+  int sched_slot;
   int causal, o_f32;
   float scale_log2;        // softmax: scale * log2(e)
   float hstu_half_alpha;   // HSTU: 0.5 * alpha      (tanh argument scale)
@@ -68,13 +92,18 @@ struct PrefillParams {
   long long wait_ns;
 };
 
+// One work item as the producer publishes it to the other roles.
+struct PfItem {
+  int bh, h, seq_start, L;  // dense: bh; packed: head and first packed row of the sequence; rows L
+  int r0;                   // first query row of the item (tile t starts at r0 + 128 t)
+  int n0, n1;               // key tiles seen by Q tile 0 / 1
+  int stop;                 // no more work
+};
+
 template <int D>
 struct PfCfg {
-  // TMEM (512 columns): S_t at 128 t, O_t at 256 + D t.  With D = 64 there is room for a separate P_t
-  // (at 384 + 64 t), so the next key tile's S_t can be computed while the softmax still works on P_t.
-  // With D = 128 TMEM is full and P_t overwrites the first 64 columns of S_t (S_t of the next key tile is
-  // then issued only after the PV that reads P_t has completed).
   static constexpr bool ALIAS_P = (D == 128);
+  static constexpr int N_ISSUERS = ALIAS_P ? 1 : 2;
   static constexpr int KCH = D / 64;                     // 128-byte column chunks per row
   static constexpr int CHUNK_BYTES = PF_BM * 128;        // 128 rows x 128 B
   static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // one 128 x D bf16 tile
@@ -82,263 +111,338 @@ struct PfCfg {
   // Of every 8 exp2 pairs, how many use the FMA-pipe polynomial instead of the MUFU.  Off: measured inside
   // this kernel it costs more (issue slots, dependency chains) than the MUFU time it saves.
   static constexpr int POLY_PAIRS = 0;
-  // barriers: full/empty per stage, q, per tile {s_full, s_free, p_full, pv_done, mma_done}
-  static constexpr int NBAR = 2 * NST + 1 + 2 * 5;
-  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + (2 + NST) * TILE_BYTES + NBAR * 8 + 16;
+  // barriers: full/empty per stage; q_full, q_empty; item_full[2], item_empty[2];
+  // per tile {s_full, s_free, p_full, pv_done, o_free, mma_done}
+  static constexpr int NBAR = 2 * NST + 2 + 4 + 2 * 6;
+  static constexpr int SMEM_BYTES =
+      1024 /*alignment slack*/ + (2 + NST) * TILE_BYTES + NBAR * 8 + 2 * (int)sizeof(PfItem) + 16;
   static constexpr uint32_t TM_O = 256;                  // O_t at TM_O + D*t
   static constexpr uint32_t TM_P = 384;                  // P_t at TM_P + 64*t (D = 64); S_t's columns [0,64) (D = 128)
 };
 
-// Control warpgroup: warp 0 streams Q, K, V with TMA; warps 1 and 2 issue the MMAs of Q tiles 0 and 1;
-// warp 3 has no role.
+// Shared-memory carve-up, common to every role.  Every member is the base address plus a compile-time
+// offset, computed where it is used (nothing but the base stays live in registers).
+template <int D>
+struct PfSmem {
+  using C = PfCfg<D>;
+  static constexpr int OFF_KV = 2 * C::TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + C::NST * C::TILE_BYTES;
+  static constexpr int B_FULL = 0, B_EMPTY = C::NST, B_QFULL = 2 * C::NST, B_QEMPTY = B_QFULL + 1,
+                       B_ITEM_FULL = B_QEMPTY + 1, B_ITEM_EMPTY = B_ITEM_FULL + 2, B_S_FULL = B_ITEM_EMPTY + 2,
+                       B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 2,
+                       B_O_FREE = B_PV_DONE + 2, B_MMA_DONE = B_O_FREE + 2, B_END = B_MMA_DONE + 2;
+  static_assert(B_END == C::NBAR, "barrier count");
+  static constexpr int OFF_ITEMS = OFF_BAR + C::NBAR * 8;
+  static constexpr int OFF_TMEM_SLOT = OFF_ITEMS + 2 * (int)sizeof(PfItem);
+  static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
+  uint8_t *base;
+  __device__ explicit PfSmem(uint8_t *smem) : base(smem) {}
+  __device__ __forceinline__ uint64_t *bar(int i) const { return reinterpret_cast<uint64_t *>(base + OFF_BAR) + i; }
+  __device__ __forceinline__ uint8_t *sQ() const { return base; }
+  __device__ __forceinline__ uint8_t *sKV() const { return base + OFF_KV; }
+  __device__ __forceinline__ uint64_t *full(int i) const { return bar(B_FULL + i); }          // TMA -> MMA
+  __device__ __forceinline__ uint64_t *empty(int i) const { return bar(B_EMPTY + i); }        // MMA -> TMA
+  // Q tiles of the current item landed / every QK^T of the item completed (Q may be overwritten)
+  __device__ __forceinline__ uint64_t *q_full() const { return bar(B_QFULL); }
+  __device__ __forceinline__ uint64_t *q_empty() const { return bar(B_QEMPTY); }
+  // item ring: published by the producer / read by every consumer warp
+  __device__ __forceinline__ uint64_t *item_full(int i) const { return bar(B_ITEM_FULL + i); }
+  __device__ __forceinline__ uint64_t *item_empty(int i) const { return bar(B_ITEM_EMPTY + i); }
+  // per Q tile t: S_t ready in TMEM (MMA -> softmax) / S_t copied to registers (softmax -> MMA; D = 64)
+  __device__ __forceinline__ uint64_t *s_full(int t) const { return bar(B_S_FULL + t); }
+  __device__ __forceinline__ uint64_t *s_free(int t) const { return bar(B_S_FREE + t); }
+  // P_t written, O_t rescaled (softmax -> MMA) / O_t += P_t V complete (MMA -> softmax)
+  __device__ __forceinline__ uint64_t *p_full(int t) const { return bar(B_P_FULL + t); }
+  __device__ __forceinline__ uint64_t *pv_done(int t) const { return bar(B_PV_DONE + t); }
+  // epilogue has read O_t (softmax -> MMA) / every MMA of issuer 1+t complete
+  __device__ __forceinline__ uint64_t *o_free(int t) const { return bar(B_O_FREE + t); }
+  __device__ __forceinline__ uint64_t *mma_done(int t) const { return bar(B_MMA_DONE + t); }
+  __device__ __forceinline__ PfItem *items() const { return reinterpret_cast<PfItem *>(base + OFF_ITEMS); }
+  __device__ __forceinline__ uint32_t *tmem_slot() const { return reinterpret_cast<uint32_t *>(base + OFF_TMEM_SLOT); }
+  __device__ __forceinline__ volatile int *abort_flag() const {
+    return reinterpret_cast<volatile int *>(base + OFF_ABORT);
+  }
+};
+
+// Work item `idx`, heaviest first: the latest row block of every (batch|sequence, head) comes first.
+template <int MODE>
+__device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int idx) {
+  PfItem it{};
+  int blk;
+  if constexpr (MODE != MODE_DENSE) {
+    const int per = p.S * p.H;
+    blk = p.nblk - 1 - idx / per;
+    const int rem = idx - (idx / per) * per;
+    const int s = rem / p.H;
+    it.h = rem - s * p.H;
+    it.seq_start = p.cu_seqlens[s];
+    it.L = p.cu_seqlens[s + 1] - it.seq_start;
+    if (it.L < 0 || it.L > p.max_len) {
+      if (blk == 0 && it.h == 0) record_status(3 /* ETA_DEV_BAD_CUSEQ */);
+      it.L = 0;  // the sequence is skipped
+    }
+  } else {
+    blk = p.nblk - 1 - idx / p.BH;
+    it.bh = idx - (idx / p.BH) * p.BH;
+    it.L = p.N;
+  }
+  it.r0 = blk * 2 * PF_BM;
+  const bool causal = (MODE == MODE_HSTU) ? true : (p.causal != 0);
+  const int qs0 = it.r0, qs1 = it.r0 + PF_BM;
+  const int e0 = (qs0 >= it.L) ? 0 : (causal ? min(it.L, qs0 + PF_BM) : it.L);
+  const int e1 = (qs1 >= it.L) ? 0 : (causal ? min(it.L, qs1 + PF_BM) : it.L);
+  it.n0 = (e0 + PF_BN - 1) / PF_BN;
+  it.n1 = (e1 + PF_BN - 1) / PF_BN;
+  it.stop = 0;
+  return it;
+}
+
+// Control warpgroup: warp 0 fetches items and streams Q, K, V with TMA; warps 1-2 issue MMAs; warp 3 idles.
 template <int D, int MODE>
 __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CUtensorMap &tmK,
                                                 const CUtensorMap &tmV, const PrefillParams &p, uint8_t *smem,
-                                                uint32_t tmem, int warp, int lane, int r0, int h, int bh,
-                                                int seq_start, const int (&n_t)[2], int n_kv) {
+                                                uint32_t tmem, int warp, int lane) {
   using C = PfCfg<D>;
-  constexpr bool HSTU = (MODE == MODE_HSTU);
   constexpr bool PACKED = (MODE != MODE_DENSE);
-  uint8_t *sQ = smem;
-  uint8_t *sKV = smem + 2 * C::TILE_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + C::NST * C::TILE_BYTES);
-  uint64_t *full = bars;
-  uint64_t *empty = bars + C::NST;
-  uint64_t *q_full = bars + 2 * C::NST;
-  uint64_t *s_full = q_full + 1;
-  uint64_t *s_free = s_full + 2;
-  uint64_t *p_full = s_free + 2;
-  uint64_t *pv_done = p_full + 2;
-  uint64_t *mma_done = pv_done + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 2);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  (void)sQ; (void)sKV; (void)full; (void)empty; (void)q_full; (void)s_full; (void)s_free;
-  (void)p_full; (void)pv_done; (void)mma_done; (void)abort_flag; (void)HSTU; (void)PACKED;
+  PfSmem<D> sm(smem);
   if (warp == 0) {
-    // ================================================================ TMA producer
+    // ================================================================ work fetcher + TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(q_full, 2 * C::TILE_BYTES);
+      int kv_issued = 0;  // K/V ring loads issued, over all items
+      int q_issued = 0;   // items whose Q tiles were loaded
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        PfItem it;
+        for (bool first = (k == 0);; first = false) {
+          // The first item of every CTA is its block index; later ones come from the shared counter.
+          const unsigned int idx = first ? blockIdx.x : gridDim.x + atomicAdd(&g_pf_sched[p.sched_slot][0], 1u);
+          if (idx >= (unsigned int)p.n_items) {
+            it = PfItem{};
+            it.stop = 1;
+            break;
+          }
+          it = decode_item<MODE>(p, (int)idx);
+          if (it.r0 < it.L) break;  // row blocks past the end of their sequence have no work
+        }
+        ok = mbar_wait(sm.item_empty(k & 1), ((k >> 1) & 1) ^ 1, sm.abort_flag(), p.wait_ns);
+        if (!ok) break;
+        sm.items()[k & 1] = it;
+        mbar_arrive(sm.item_full(k & 1));  // release semantics: the item is visible to its readers
+        if (it.stop) break;
+        // Q tiles: every QK^T of the previous item must have finished reading them.
+        if (k > 0) {
+          ok = mbar_wait(sm.q_empty(), (k - 1) & 1, sm.abort_flag(), p.wait_ns);
+          if (!ok) break;
+        }
+        mbar_arrive_expect_tx(sm.q_full(), 2 * C::TILE_BYTES);
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < 2; ++t) {
 #pragma unroll
-        for (int c = 0; c < C::KCH; ++c) {
-          uint8_t *dst = sQ + t * C::TILE_BYTES + c * C::CHUNK_BYTES;
-          if constexpr (PACKED)
-            tma_load_3d(dst, &tmQ, q_full, 64 * c, h, seq_start + r0 + t * PF_BM);
-          else
-            tma_load_3d(dst, &tmQ, q_full, 64 * c, r0 + t * PF_BM, bh);
+          for (int c = 0; c < C::KCH; ++c) {
+            uint8_t *dst = sm.sQ() + t * C::TILE_BYTES + c * C::CHUNK_BYTES;
+            if constexpr (PACKED)
+              tma_load_3d(dst, &tmQ, sm.q_full(), 64 * c, it.h, it.seq_start + it.r0 + t * PF_BM);
+            else
+              tma_load_3d(dst, &tmQ, sm.q_full(), 64 * c, it.r0 + t * PF_BM, it.bh);
+          }
+        }
+        ++q_issued;
+        const int n_loads = 2 * max(it.n0, it.n1);
+        for (int i = 0; i < n_loads; ++i) {
+          const int st = kv_issued % C::NST;
+          ok = mbar_wait(sm.empty(st), ((kv_issued / C::NST) & 1) ^ 1, sm.abort_flag(), p.wait_ns);
+          if (!ok) break;
+          const int j = i >> 1;
+          const CUtensorMap *m = (i & 1) ? &tmV : &tmK;
+          mbar_arrive_expect_tx(sm.full(st), C::TILE_BYTES);
+#pragma unroll
+          for (int c = 0; c < C::KCH; ++c) {
+            uint8_t *dst = sm.sKV() + st * C::TILE_BYTES + c * C::CHUNK_BYTES;
+            if constexpr (PACKED)
+              tma_load_3d(dst, m, sm.full(st), 64 * c, it.h, it.seq_start + j * PF_BN);
+            else
+              tma_load_3d(dst, m, sm.full(st), 64 * c, j * PF_BN, it.bh);
+          }
+          ++kv_issued;
         }
       }
-      int item = 0;
-      const int n_items = 2 * n_kv;
-      for (; item < n_items; ++item) {
-        const int st = item % C::NST;
-        if (!mbar_wait(&empty[st], ((item / C::NST) & 1) ^ 1, abort_flag, p.wait_ns)) break;
-        const int j = item >> 1;
-        const CUtensorMap *m = (item & 1) ? &tmV : &tmK;
-        mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
-#pragma unroll
-        for (int c = 0; c < C::KCH; ++c) {
-          uint8_t *dst = sKV + st * C::TILE_BYTES + c * C::CHUNK_BYTES;
-          if constexpr (PACKED)
-            tma_load_3d(dst, m, &full[st], 64 * c, h, seq_start + j * PF_BN);
-          else
-            tma_load_3d(dst, m, &full[st], 64 * c, j * PF_BN, bh);
-        }
-      }
-      if (item < n_items) {
+      if (!ok) {
         // Abandoned pipeline: let copies already in flight land before shared memory is released.
-        mbar_wait(q_full, 0, nullptr, p.wait_ns);
-        for (int i = max(0, item - C::NST); i < item; ++i)
-          mbar_wait(&full[i % C::NST], (i / C::NST) & 1, nullptr, p.wait_ns);
+        if (q_issued > 0) mbar_wait(sm.q_full(), (q_issued - 1) & 1, nullptr, p.wait_ns);
+        for (int i = max(0, kv_issued - C::NST); i < kv_issued; ++i)
+          mbar_wait(sm.full(i % C::NST), (i / C::NST) & 1, nullptr, p.wait_ns);
       }
     }
-  } else if (C::ALIAS_P && warp == 1) {
-    // ================================================================ single MMA issuer (P aliased into S)
-    // One thread issues both tiles' MMAs in the order PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  tcgen05.mma
-    // operations issued by one thread execute in issue order, so S_t(j+1) -- which overwrites the columns
-    // holding P_t(j) -- needs no wait for PV_t(j) to complete; its commit also tracks that PV, so a softmax
-    // that has seen S_t(j+1) may rescale O_t.  The single ordered stream keeps the two softmax warpgroups
-    // half a period apart.
+  } else if (warp == 1 || (!C::ALIAS_P && warp == 2)) {
+    // ================================================================ MMA issuer(s)
     if (lane == 0) {
       constexpr uint32_t ID_QK = idesc_bf16_f32(PF_BM, PF_BN, false);
       constexpr uint32_t ID_PV = idesc_bf16_f32(PF_BM, D, true);
-      const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
+      const uint32_t sQa = smem_u32(sm.sQ()), sKVa = smem_u32(sm.sKV());
+      // S_t = Q_t K^T : K-steps of 16 elements = 32 bytes inside a 128-byte swizzled row.
+      const uint64_t dQ = sdesc_sw128(sQa, 16, 1024), dKV = sdesc_sw128(sKVa, 16, 1024);
+      const uint64_t dV = sdesc_sw128(sKVa, C::CHUNK_BYTES, 1024);
       auto issue_s = [&](int t, int st) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)(kk >> 2) * C::CHUNK_BYTES + (uint32_t)(kk & 3) * 32u;
-          mma_ss(tmem + 128u * t, sdesc_sw128(sQa + t * C::TILE_BYTES + off, 16, 1024),
-                 sdesc_sw128(sKVa + st * C::TILE_BYTES + off, 16, 1024), ID_QK, kk > 0 ? 1u : 0u);
-        }
+        const uint64_t da = dQ + (uint64_t)((t * C::TILE_BYTES) >> 4);
+        const uint64_t db = dKV + (uint64_t)((st * C::TILE_BYTES) >> 4);
+        const uint32_t dt = tmem + 128u * t;
+        eta_static_for<D / 16>([&](auto kk_c) {
+          constexpr int kk = decltype(kk_c)::value;
+          constexpr uint32_t off = ((uint32_t)(kk >> 2) * C::CHUNK_BYTES + (uint32_t)(kk & 3) * 32u) >> 4;
+          mma_ss_off<off, off>(dt, da, db, ID_QK, kk > 0 ? 1u : 0u);
+        });
       };
+      // O_t += P_t V : K-steps of 16 keys = 8 TMEM columns of packed bf16 P, 16 rows (2048 B) of V.
       auto issue_pv = [&](int t, int st, bool acc) {
-#pragma unroll
-        for (int kk = 0; kk < PF_BN / 16; ++kk)
-          mma_ts(tmem + C::TM_O + (uint32_t)(D * t), tmem + 128u * t + 8u * kk,
-                 sdesc_sw128(sKVa + st * C::TILE_BYTES + kk * 2048, C::CHUNK_BYTES, 1024), ID_PV,
-                 (acc || kk > 0) ? 1u : 0u);
+        const uint32_t tP = C::ALIAS_P ? tmem + 128u * t : tmem + C::TM_P + 64u * t;
+        const uint64_t db = dV + (uint64_t)((st * C::TILE_BYTES) >> 4);
+        const uint32_t dt = tmem + C::TM_O + (uint32_t)(D * t);
+        const uint32_t acc0 = acc ? 1u : 0u;
+        eta_static_for<PF_BN / 16>([&](auto kk_c) {
+          constexpr int kk = decltype(kk_c)::value;
+          constexpr uint32_t ta_off = 8u * kk, b_off = (2048u * kk) / 16u;
+          mma_ts_off<ta_off, b_off>(dt, tP, db, ID_PV, kk > 0 ? 1u : acc0);
+        });
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.wait_ns);
-      if (ok && n_kv > 0) {
-        ok = mbar_wait(&full[0], 0, abort_flag, p.wait_ns);
-        if (ok) {
+      // Counts over all items; each gives the phase of the barrier it tracks.  With one issuer per tile
+      // only slot 0 is used (for the issuer's own tile).
+      int gs[2] = {0, 0};  // QK^T issued for tile t           (s_full / s_free completions)
+      int gp[2] = {0, 0};  // PV issued for tile t             (p_full / pv_done completions)
+      int go[2] = {0, 0};  // items with rows in tile t        (o_free completions)
+      int kv_base = 0;     // ring index of the current item's K_0
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        ok = mbar_wait(sm.item_full(k & 1), (k >> 1) & 1, sm.abort_flag(), p.wait_ns);
+        if (!ok) break;
+        const PfItem it = sm.items()[k & 1];
+        mbar_arrive(sm.item_empty(k & 1));
+        if (it.stop) break;
+        const int n_t[2] = {it.n0, it.n1};
+        const int n_kv = max(it.n0, it.n1);  // >= 1: an item has at least one row
+        ok = mbar_wait(sm.q_full(), k & 1, sm.abort_flag(), p.wait_ns);
+        if (!ok) break;
+        // K/V ring: K_j is item-local load 2j, V_j is 2j + 1.
+        auto kv_wait = [&](int i) {
+          const int g = kv_base + i;
+          return mbar_wait(sm.full(g % C::NST), (g / C::NST) & 1, sm.abort_flag(), p.wait_ns);
+        };
+        auto kv_stage = [&](int i) { return (kv_base + i) % C::NST; };
+        // Before the first PV of an item overwrites O_t, the previous item's epilogue must have read it.
+        // (c: the counter slot of tile t -- t itself with one issuer, 0 for a per-tile issuer.)
+        auto o_wait = [&](int t, int c) {
+          return go[c] == 0 || mbar_wait(sm.o_free(t), (go[c] - 1) & 1, sm.abort_flag(), p.wait_ns);
+        };
+        if constexpr (!C::ALIAS_P) {
+          // ---------------- issuer 1+t serves Q tile t; the next S_t as soon as S_t is free
+          const int t = warp - 1;
+          const int nt = (t == 0) ? it.n0 : it.n1;
+          if (nt > 0) {
+            ok = kv_wait(0) && (gs[0] == 0 || mbar_wait(sm.s_free(t), (gs[0] - 1) & 1, sm.abort_flag(), p.wait_ns));
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(t, kv_stage(0));
+            mma_commit(sm.s_full(t));
+            mma_commit(sm.empty(kv_stage(0)));
+            ++gs[0];
+          }
+          if (nt <= 1) mma_commit(sm.q_empty());  // every QK^T of this item is issued
+          for (int j = 0; ok && j < nt; ++j) {
+            if (j + 1 < nt) {
+              ok = kv_wait(2 * j + 2) && mbar_wait(sm.s_free(t), (gs[0] - 1) & 1, sm.abort_flag(), p.wait_ns);
+              if (!ok) break;
+              tc_fence_after();
+              issue_s(t, kv_stage(2 * j + 2));
+              mma_commit(sm.s_full(t));
+              mma_commit(sm.empty(kv_stage(2 * j + 2)));
+              ++gs[0];
+              if (j + 2 == nt) mma_commit(sm.q_empty());
+            }
+            ok = kv_wait(2 * j + 1) && mbar_wait(sm.p_full(t), gp[0] & 1, sm.abort_flag(), p.wait_ns) &&
+                 (j > 0 || o_wait(t, 0));
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, kv_stage(2 * j + 1), j > 0);
+            mma_commit(sm.pv_done(t));
+            mma_commit(sm.empty(kv_stage(2 * j + 1)));
+            ++gp[0];
+          }
+          // Key/value tiles of this item that tile t does not see: release them once they landed.
+          for (int i = 2 * nt; ok && i < 2 * n_kv; ++i) {
+            ok = kv_wait(i);
+            if (ok) mbar_arrive(sm.empty(kv_stage(i)));
+          }
+          if (nt > 0) ++go[0];
+        } else {
+          // ---------------- one issuer for both tiles; P aliased into S; issue order PV_t(j), S_t(j+1)
+          ok = kv_wait(0);
+          if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int t = 0; t < 2; ++t)
             if (n_t[t] > 0) {
-              issue_s(t, 0);
-              mma_commit(&s_full[t]);
+              issue_s(t, kv_stage(0));
+              mma_commit(sm.s_full(t));
+              ++gs[t];
             }
-          mma_commit(&empty[0]);
-        }
-      }
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int iv = 2 * j + 1, sv = iv % C::NST;
-        const int ik = 2 * j + 2, sk = ik % C::NST;
-        ok = mbar_wait(&full[sv], (iv / C::NST) & 1, abort_flag, p.wait_ns);
-        if (!ok) break;
-        bool k_ready = false;
+          mma_commit(sm.empty(kv_stage(0)));
+          if (n_kv == 1) mma_commit(sm.q_empty());
+          for (int j = 0; ok && j < n_kv; ++j) {
+            ok = kv_wait(2 * j + 1);
+            if (!ok) break;
+            bool k_ready = false;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (!ok || j >= n_t[t]) continue;
-          ok = mbar_wait(&p_full[t], j & 1, abort_flag, p.wait_ns);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(t, sv, j > 0);
-          mma_commit(&pv_done[t]);
-          if (j + 1 < n_t[t]) {
-            if (!k_ready) {
-              ok = mbar_wait(&full[sk], (ik / C::NST) & 1, abort_flag, p.wait_ns);
+            for (int t = 0; t < 2; ++t) {
+              if (!ok || j >= n_t[t]) continue;
+              ok = mbar_wait(sm.p_full(t), gp[t] & 1, sm.abort_flag(), p.wait_ns) && (j > 0 || o_wait(t, t));
               if (!ok) break;
-              k_ready = true;
+              tc_fence_after();
+              issue_pv(t, kv_stage(2 * j + 1), j > 0);
+              mma_commit(sm.pv_done(t));
+              ++gp[t];
+              if (j + 1 < n_t[t]) {
+                if (!k_ready) {
+                  ok = kv_wait(2 * j + 2);
+                  if (!ok) break;
+                  k_ready = true;
+                }
+                issue_s(t, kv_stage(2 * j + 2));
+                mma_commit(sm.s_full(t));
+                ++gs[t];
+              }
             }
-            issue_s(t, sk);
-            mma_commit(&s_full[t]);
-          }
-        }
-        if (!ok) break;
-        mma_commit(&empty[sv]);
-        if (k_ready) mma_commit(&empty[sk]);
-      }
-      mma_commit(&mma_done[0]);
-      mbar_wait(&mma_done[0], 0, nullptr, p.wait_ns);
-    }
-    __syncwarp();
-  } else if (!C::ALIAS_P && (warp == 1 || warp == 2)) {
-    // ================================================================ MMA issuer for Q tile t
-    const int t = warp - 1;
-    if (lane == 0) {
-      constexpr uint32_t ID_QK = idesc_bf16_f32(PF_BM, PF_BN, false);
-      constexpr uint32_t ID_PV = idesc_bf16_f32(PF_BM, D, true);
-      const uint32_t sQa = smem_u32(sQ) + t * C::TILE_BYTES, sKVa = smem_u32(sKV);
-      const uint32_t tS = tmem + 128u * t, tO = tmem + C::TM_O + (uint32_t)(D * t);
-      const uint32_t tP = C::ALIAS_P ? tS : tmem + C::TM_P + 64u * t;
-      // S_t = Q_t K^T : K-steps of 16 elements = 32 bytes inside a 128-byte swizzled row.
-      auto issue_s = [&](int st) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)(kk >> 2) * C::CHUNK_BYTES + (uint32_t)(kk & 3) * 32u;
-          mma_ss(tS, sdesc_sw128(sQa + off, 16, 1024), sdesc_sw128(sKVa + st * C::TILE_BYTES + off, 16, 1024), ID_QK,
-                 kk > 0 ? 1u : 0u);
-        }
-      };
-      // O_t += P_t V : K-steps of 16 keys = 8 TMEM columns of packed bf16 P, 16 rows (2048 B) of V.
-      auto issue_pv = [&](int st, bool acc) {
-#pragma unroll
-        for (int kk = 0; kk < PF_BN / 16; ++kk)
-          mma_ts(tO, tP + 8u * kk, sdesc_sw128(sKVa + st * C::TILE_BYTES + kk * 2048, C::CHUNK_BYTES, 1024), ID_PV,
-                 (acc || kk > 0) ? 1u : 0u);
-      };
-      const int nt = n_t[t];
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.wait_ns);
-      if (ok && nt > 0) {
-        ok = mbar_wait(&full[0], 0, abort_flag, p.wait_ns);
-        if (ok) {
-          tc_fence_after();
-          issue_s(0);
-          mma_commit(&s_full[t]);
-          mma_commit(&empty[0]);
-        }
-      }
-      for (int j = 0; ok && j < nt; ++j) {
-        const int ik = 2 * j + 2, sk = ik % C::NST;
-        const int iv = 2 * j + 1, sv = iv % C::NST;
-        if constexpr (!C::ALIAS_P) {
-          // Separate P: S_t of the next key tile as soon as the softmax has copied S_t to registers.
-          if (j + 1 < nt) {
-            ok = mbar_wait(&full[sk], (ik / C::NST) & 1, abort_flag, p.wait_ns) &&
-                 mbar_wait(&s_free[t], j & 1, abort_flag, p.wait_ns);
             if (!ok) break;
-            tc_fence_after();
-            issue_s(sk);
-            mma_commit(&s_full[t]);
-            mma_commit(&empty[sk]);
+            mma_commit(sm.empty(kv_stage(2 * j + 1)));
+            if (k_ready) mma_commit(sm.empty(kv_stage(2 * j + 2)));
+            if (j + 2 == n_kv) mma_commit(sm.q_empty());
           }
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if (n_t[t] > 0) ++go[t];
         }
-        ok = mbar_wait(&full[sv], (iv / C::NST) & 1, abort_flag, p.wait_ns) &&
-             mbar_wait(&p_full[t], j & 1, abort_flag, p.wait_ns);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(sv, j > 0);
-        mma_commit(&pv_done[t]);
-        mma_commit(&empty[sv]);
-        if constexpr (C::ALIAS_P) {
-          // P_t lives in S_t's columns: the PV just issued must finish reading it first.
-          if (j + 1 < nt) {
-            ok = mbar_wait(&full[sk], (ik / C::NST) & 1, abort_flag, p.wait_ns) &&
-                 mbar_wait(&pv_done[t], j & 1, abort_flag, p.wait_ns);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(sk);
-            mma_commit(&s_full[t]);
-            mma_commit(&empty[sk]);
-          }
-        }
-      }
-      // Key/value tiles this Q tile does not see (past its diagonal, or the whole tile past the end):
-      // release them too, in order, once they have landed.
-      for (int item = 2 * nt; ok && item < 2 * n_kv; ++item) {
-        ok = mbar_wait(&full[item % C::NST], (item / C::NST) & 1, abort_flag, p.wait_ns);
-        if (ok) mbar_arrive(&empty[item % C::NST]);
+        kv_base += 2 * n_kv;
       }
       // Every MMA issued by this thread has completed before TMEM is released.
-      mma_commit(&mma_done[t]);
-      mbar_wait(&mma_done[t], 0, nullptr, p.wait_ns);
+      mma_commit(sm.mma_done(warp - 1));
+      mbar_wait(sm.mma_done(warp - 1), 0, nullptr, p.wait_ns);
     }
     __syncwarp();
   }
 }
 
 // Softmax (or HSTU pointwise) warpgroups: warps 4-7 for Q tile 0, warps 8-11 for Q tile 1.  Thread
-// (quarter, lane) owns query row 32 quarter + lane of its tile (= its TMEM lane): it loads the S row from
-// TMEM, applies the mask, updates the running max and exp-sum, writes P (bf16) to TMEM, rescales its O row
-// when the max moved, and finally normalises O and stores O and lse.
+// (quarter, lane) owns query row 32 quarter + lane of its tile (= its TMEM lane): per key tile it loads the
+// S row from TMEM, applies the mask, updates the running max and exp-sum, writes P (bf16) to TMEM and
+// rescales its O row when the max moved; per item it finally normalises O and stores O and lse.
 template <int D, int MODE>
 __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t *smem, uint32_t tmem, int warp,
-                                                int lane, int r0, int L, int h, int bh, int seq_start, bool causal,
-                                                const int (&n_t)[2]) {
+                                                int lane) {
   using C = PfCfg<D>;
   constexpr bool HSTU = (MODE == MODE_HSTU);
   constexpr bool PACKED = (MODE != MODE_DENSE);
-  uint8_t *sQ = smem;
-  uint8_t *sKV = smem + 2 * C::TILE_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + C::NST * C::TILE_BYTES);
-  uint64_t *full = bars;
-  uint64_t *empty = bars + C::NST;
-  uint64_t *q_full = bars + 2 * C::NST;
-  uint64_t *s_full = q_full + 1;
-  uint64_t *s_free = s_full + 2;
-  uint64_t *p_full = s_free + 2;
-  uint64_t *pv_done = p_full + 2;
-  uint64_t *mma_done = pv_done + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 2);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  (void)sQ; (void)sKV; (void)full; (void)empty; (void)q_full; (void)s_full; (void)s_free;
-  (void)p_full; (void)pv_done; (void)mma_done; (void)abort_flag; (void)HSTU; (void)PACKED;
+  PfSmem<D> sm(smem);
   const int t = (warp - 4) >> 2;
   const int quarter = warp & 3;
   const int row = quarter * 32 + lane;
@@ -346,155 +450,172 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
   const uint32_t tS = tmem + lane_addr + 128u * t;
   const uint32_t tO = tmem + lane_addr + C::TM_O + (uint32_t)(D * t);
   const uint32_t tP = C::ALIAS_P ? tS : tmem + lane_addr + C::TM_P + 64u * t;
-  const int q_start = r0 + t * PF_BM;
-  const int qpos = q_start + row;
-  const int nt = n_t[t];
-  float m_used = -INFINITY, l = 0.f;
+  const bool causal = HSTU ? true : (p.causal != 0);
+  int gj = 0;  // key tiles of Q tile t processed, over all items (phases of s_full, p_full, pv_done)
   bool ok = true;
-  for (int j = 0; j < nt; ++j) {
-    ok = mbar_wait(&s_full[t], j & 1, abort_flag, p.wait_ns);
+  for (int k = 0; ok; ++k) {
+    ok = mbar_wait(sm.item_full(k & 1), (k >> 1) & 1, sm.abort_flag(), p.wait_ns);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    const PfItem it = sm.items()[k & 1];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.item_empty(k & 1));
+    if (it.stop) break;
+    const int L = it.L;
+    const int q_start = it.r0 + t * PF_BM;
+    const int qpos = q_start + row;
+    const int nt = (t == 0) ? it.n0 : it.n1;
+    float m_used = -INFINITY, l = 0.f;
+    for (int j = 0; j < nt; ++j, ++gj) {
+      ok = mbar_wait(sm.s_full(t), gj & 1, sm.abort_flag(), p.wait_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[128];
+      ETA_TMEM_LD_X32(tS + 0u, (sr + 0));
+      ETA_TMEM_LD_X32(tS + 32u, (sr + 32));
+      ETA_TMEM_LD_X32(tS + 64u, (sr + 64));
+      ETA_TMEM_LD_X32(tS + 96u, (sr + 96));
+      tmem_wait_ld();
+      if constexpr (!C::ALIAS_P) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sm.s_free(t));  // S_t may now be overwritten by the next QK^T
+      }
+      const int k0 = j * PF_BN;
+      const bool need_mask = (k0 + PF_BN > L) || (causal && k0 + PF_BN - 1 > q_start);
+      const int kmax = causal ? min(L - 1, qpos) - k0 : L - 1 - k0;  // last visible key, tile-local
+      uint32_t pk[64];
+      bool resc = false;
+      float f = 1.f, rowsum = 0.f, m_new = m_used;
+      if constexpr (!HSTU) {
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > kmax) sr[c] = __float_as_uint(-INFINITY);
+        }
+        // row max: four independent 3-input max chains
+        float mxa = -INFINITY, mxb = -INFINITY, mxc = -INFINITY, mxd = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; c += 8) {
+          mxa = max3f(mxa, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
+          mxb = max3f(mxb, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+          mxc = max3f(mxc, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+          mxd = max3f(mxd, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+        }
+        const float mx = max3f(mxa, mxb, fmaxf(mxc, mxd)) * p.scale_log2;
+        if (mx > m_used + PF_RESCALE_THRESHOLD) {
+          m_new = mx;
+          resc = true;
+        }
+        const float msub = (m_new == -INFINITY) ? 0.f : m_new;
+        const uint64_t cs2 = f2pack(p.scale_log2, p.scale_log2), nm2 = f2pack(-msub, -msub);
+        uint64_t rs_a = f2pack(0.f, 0.f), rs_b = f2pack(0.f, 0.f);
+        // p = 2^(s * scale_log2 - m): pairs with (i % 8) < POLY_PAIRS go to the FMA-pipe polynomial on
+        // unmasked tiles, the rest (and every element of a masked tile) to the MUFU.
+        auto exp_row = [&](auto use_poly) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const uint64_t x2 =
+                fma_x2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), cs2, nm2);
+            float x0, x1, p0, p1;
+            f2unpack(x2, x0, x1);
+            if (decltype(use_poly)::value && (i % 8) < C::POLY_PAIRS) {
+              exp2_poly_x2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            if (i & 1) rs_b = add_x2(rs_b, f2pack(p0, p1));
+            else rs_a = add_x2(rs_a, f2pack(p0, p1));
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+        };
+        if (need_mask) exp_row(std::false_type{});
+        else exp_row(std::true_type{});
+        float r0a, r1a, r2a, r3a;
+        f2unpack(rs_a, r0a, r1a);
+        f2unpack(rs_b, r2a, r3a);
+        rowsum = (r0a + r1a) + (r2a + r3a);
+        f = resc ? ex2_approx(m_used - msub) : 1.f;  // 0 on the first tile
+      } else {
+        // HSTU: p = inv_n * silu(alpha s) = h + h * tanh(alpha s / 2),  h = (alpha * inv_n / 2) s
+        const uint64_t ha2 = f2pack(p.hstu_half_alpha, p.hstu_half_alpha), ho2 = f2pack(p.hstu_out, p.hstu_out);
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int c0 = 2 * i;
+          const uint64_t s2 = f2pack(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1]));
+          float y0, y1;
+          f2unpack(mul_x2(s2, ha2), y0, y1);
+          const uint64_t h2 = mul_x2(s2, ho2);
+          float p0, p1;
+          f2unpack(fma_x2(h2, f2pack(tanh_approx(y0), tanh_approx(y1)), h2), p0, p1);
+          if (need_mask) {
+            p0 = (c0 > kmax) ? 0.f : p0;
+            p1 = (c0 + 1 > kmax) ? 0.f : p1;
+          }
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+      }
+      if constexpr (!C::ALIAS_P) {
+        // P_t's columns (and O_t) are free once the previous PV of this tile -- possibly the previous
+        // item's last -- has completed.  (With P aliased into S_t this is implied: the S_t just read was
+        // issued after that PV, and its commit covers it.)
+        if (gj > 0) {
+          ok = mbar_wait(sm.pv_done(t), (gj - 1) & 1, sm.abort_flag(), p.wait_ns);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+        }
+      }
+      ETA_TMEM_ST_X32(tP + 0u, (pk + 0));
+      ETA_TMEM_ST_X32(tP + 32u, (pk + 32));
+      if constexpr (!HSTU) {
+        if (__any_sync(0xffffffffu, resc && j > 0)) {
+          const uint64_t f2 = f2pack(f, f);
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t orr[32];
+            ETA_TMEM_LD_X32(tO + 32u * cc, orr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float a, b;
+              f2unpack(mul_x2(f2pack(__uint_as_float(orr[2 * i]), __uint_as_float(orr[2 * i + 1])), f2), a, b);
+              orr[2 * i] = __float_as_uint(a);
+              orr[2 * i + 1] = __float_as_uint(b);
+            }
+            ETA_TMEM_ST_X32(tO + 32u * cc, orr);
+          }
+        }
+        l = l * f + rowsum;
+        m_used = m_new;
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.p_full(t));
+    }
+    if (!ok) break;
+    if (nt == 0) continue;
+    // ---------------------------------------------------------------- epilogue of the item
+    ok = mbar_wait(sm.pv_done(t), (gj - 1) & 1, sm.abort_flag(), p.wait_ns);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     tc_fence_after();
-    uint32_t sr[128];
-    ETA_TMEM_LD_X32(tS + 0u, (sr + 0));
-    ETA_TMEM_LD_X32(tS + 32u, (sr + 32));
-    ETA_TMEM_LD_X32(tS + 64u, (sr + 64));
-    ETA_TMEM_LD_X32(tS + 96u, (sr + 96));
-    tmem_wait_ld();
-    if constexpr (!C::ALIAS_P) {
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[t]);  // S_t may now be overwritten by the next key tile's QK^T
-    }
-    const int k0 = j * PF_BN;
-    const bool need_mask = (k0 + PF_BN > L) || (causal && k0 + PF_BN - 1 > q_start);
-    const int kmax = causal ? min(L - 1, qpos) - k0 : L - 1 - k0;  // last visible key, tile-local
-    uint32_t pk[64];
-    bool resc = false;
-    float f = 1.f, rowsum = 0.f, m_new = m_used;
-    if constexpr (!HSTU) {
-      if (need_mask) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c > kmax) sr[c] = __float_as_uint(-INFINITY);
-      }
-      // row max: four independent 3-input max chains
-      float mxa = -INFINITY, mxb = -INFINITY, mxc = -INFINITY, mxd = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; c += 8) {
-        mxa = max3f(mxa, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
-        mxb = max3f(mxb, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
-        mxc = max3f(mxc, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
-        mxd = max3f(mxd, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
-      }
-      const float mx = max3f(mxa, mxb, fmaxf(mxc, mxd)) * p.scale_log2;
-      if (mx > m_used + PF_RESCALE_THRESHOLD) {
-        m_new = mx;
-        resc = true;
-      }
-      const float msub = (m_new == -INFINITY) ? 0.f : m_new;
-      const uint64_t cs2 = f2pack(p.scale_log2, p.scale_log2), nm2 = f2pack(-msub, -msub);
-      uint64_t rs_a = f2pack(0.f, 0.f), rs_b = f2pack(0.f, 0.f);
-      // p = 2^(s * scale_log2 - m): pairs with (i % 8) < POLY_PAIRS go to the FMA-pipe polynomial on
-      // unmasked tiles, the rest (and every element of a masked tile) to the MUFU.
-      auto exp_row = [&](auto use_poly) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const uint64_t x2 =
-              fma_x2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), cs2, nm2);
-          float x0, x1, p0, p1;
-          f2unpack(x2, x0, x1);
-          if (decltype(use_poly)::value && (i % 8) < C::POLY_PAIRS) {
-            exp2_poly_x2(x0, x1, p0, p1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          if (i & 1) rs_b = add_x2(rs_b, f2pack(p0, p1));
-          else rs_a = add_x2(rs_a, f2pack(p0, p1));
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-      };
-      if (need_mask) exp_row(std::false_type{});
-      else exp_row(std::true_type{});
-      float r0a, r1a, r2a, r3a;
-      f2unpack(rs_a, r0a, r1a);
-      f2unpack(rs_b, r2a, r3a);
-      rowsum = (r0a + r1a) + (r2a + r3a);
-      f = resc ? ex2_approx(m_used - msub) : 1.f;  // 0 on the first tile
-    } else {
-      // HSTU: p = inv_n * silu(alpha s) = h + h * tanh(alpha s / 2),  h = (alpha * inv_n / 2) s
-      const uint64_t ha2 = f2pack(p.hstu_half_alpha, p.hstu_half_alpha), ho2 = f2pack(p.hstu_out, p.hstu_out);
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const int c0 = 2 * i;
-        const uint64_t s2 = f2pack(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1]));
-        float y0, y1;
-        f2unpack(mul_x2(s2, ha2), y0, y1);
-        const uint64_t h2 = mul_x2(s2, ho2);
-        float p0, p1;
-        f2unpack(fma_x2(h2, f2pack(tanh_approx(y0), tanh_approx(y1)), h2), p0, p1);
-        if (need_mask) {
-          p0 = (c0 > kmax) ? 0.f : p0;
-          p1 = (c0 + 1 > kmax) ? 0.f : p1;
-        }
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-    }
-    if constexpr (!C::ALIAS_P) {
-      // P_t's buffer (and O_t) are free once the previous key tile's PV has completed.  (With P aliased into
-      // S_t this is implied: S_t of this key tile was issued only after that PV completed.)
-      if (j > 0) {
-        ok = mbar_wait(&pv_done[t], (j - 1) & 1, abort_flag, p.wait_ns);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-      }
-    }
-    ETA_TMEM_ST_X32(tP + 0u, (pk + 0));
-    ETA_TMEM_ST_X32(tP + 32u, (pk + 32));
-    if constexpr (!HSTU) {
-      if (__any_sync(0xffffffffu, resc && j > 0)) {
-        const uint64_t f2 = f2pack(f, f);
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t orr[32];
-          ETA_TMEM_LD_X32(tO + 32u * cc, orr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float a, b;
-            f2unpack(mul_x2(f2pack(__uint_as_float(orr[2 * i]), __uint_as_float(orr[2 * i + 1])), f2), a, b);
-            orr[2 * i] = __float_as_uint(a);
-            orr[2 * i + 1] = __float_as_uint(b);
-          }
-          ETA_TMEM_ST_X32(tO + 32u * cc, orr);
-        }
-      }
-      l = l * f + rowsum;
-      m_used = m_new;
-    }
-    tmem_wait_st();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&p_full[t]);
-  }
-  // ---------------------------------------------------------------- epilogue
-  if (ok && nt > 0) {
-    ok = mbar_wait(&pv_done[t], (nt - 1) & 1, abort_flag, p.wait_ns);
-    ok = __all_sync(0xffffffffu, ok);
-  }
-  if (ok && nt > 0) {
-    tc_fence_after();
     const float inv_l = HSTU ? 1.f : ((l > 0.f) ? 1.f / l : 0.f);
     const bool valid = qpos < L;
-    const size_t orow = PACKED ? ((size_t)(seq_start + qpos) * p.H + h) : ((size_t)bh * p.N + qpos);
+    const size_t orow = PACKED ? ((size_t)(it.seq_start + qpos) * p.H + it.h) : ((size_t)it.bh * p.N + qpos);
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t orr[32];
       ETA_TMEM_LD_X32(tO + 32u * cc, orr);
       tmem_wait_ld();
+      if (cc == D / 32 - 1) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sm.o_free(t));  // the next item's first PV may overwrite O_t
+      }
       if (valid) {
         if (p.o_f32) {
           float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D + 32 * cc);
@@ -516,9 +637,10 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
         }
       }
     }
-    if constexpr (!HSTU) {
-      if (valid && p.lse != nullptr)
-        p.lse[orow] = (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    if (valid) {
+      if constexpr (!HSTU) {
+        if (p.lse != nullptr) p.lse[orow] = (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      }
     }
   }
 }
@@ -528,94 +650,66 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   using C = PfCfg<D>;
-  constexpr bool HSTU = (MODE == MODE_HSTU);
-  constexpr bool PACKED = (MODE != MODE_DENSE);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQ = smem;                                        // 2 tiles
-  uint8_t *sKV = smem + 2 * C::TILE_BYTES;                   // NST tiles
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + C::NST * C::TILE_BYTES);
-  uint64_t *full = bars;                 // [NST] TMA -> MMA issuers
-  uint64_t *empty = bars + C::NST;       // [NST] both MMA issuers -> TMA (count 2)
-  uint64_t *q_full = bars + 2 * C::NST;  // Q tiles landed
-  uint64_t *s_full = q_full + 1;         // [2] S_t ready in TMEM              (MMA t -> softmax t)
-  uint64_t *s_free = s_full + 2;         // [2] S_t copied to registers        (softmax t -> MMA t; D = 64)
-  uint64_t *p_full = s_free + 2;         // [2] P_t written, O_t rescaled      (softmax t -> MMA t)
-  uint64_t *pv_done = p_full + 2;        // [2] O_t += P_t V complete           (MMA t -> softmax t, MMA t)
-  uint64_t *mma_done = pv_done + 2;      // [2] every MMA of issuer t complete
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 2);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-
+  PfSmem<D> sm(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // ------------------------------------------------------------------ work item
-  // Heaviest (latest) row blocks are launched first: dense grid (B*H, blocks), packed grid (H, S, blocks).
-  const int blk = PACKED ? (int)(gridDim.z - 1 - blockIdx.z) : (int)(gridDim.y - 1 - blockIdx.y);
-  int L, seq_start = 0, bh = 0, h = 0;
-  if constexpr (PACKED) {
-    h = blockIdx.x;
-    const int s = blockIdx.y;
-    seq_start = p.cu_seqlens[s];
-    L = p.cu_seqlens[s + 1] - seq_start;
-    if (L < 0 || L > p.max_len) {
-      if (threadIdx.x == 0 && blk == 0) record_status(3 /* ETA_DEV_BAD_CUSEQ */);
-      return;
-    }
-  } else {
-    bh = blockIdx.x;
-    L = p.N;
-  }
-  const int r0 = blk * 2 * PF_BM;
-  if (r0 >= L) return;  // uniform over the CTA
-  const bool causal = HSTU ? true : (p.causal != 0);
-  int n_t[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int qs = r0 + t * PF_BM;
-    const int kv_end = (qs >= L) ? 0 : (causal ? min(L, qs + PF_BM) : L);
-    n_t[t] = (kv_end + PF_BN - 1) / PF_BN;
-  }
-  const int n_kv = max(n_t[0], n_t[1]);
 
   // ------------------------------------------------------------------ setup
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], C::ALIAS_P ? 1 : 2);  // released by each MMA issuer
+      mbar_init(sm.full(i), 1);
+      mbar_init(sm.empty(i), C::N_ISSUERS);  // released by each MMA issuer
     }
-    mbar_init(q_full, 1);
+    mbar_init(sm.q_full(), 1);
+    mbar_init(sm.q_empty(), C::N_ISSUERS);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(sm.item_full(i), 1);
+      mbar_init(sm.item_empty(i), C::N_ISSUERS + PF_SM_WARPS);  // every consumer warp reads the item
+    }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&s_full[t], 1);
-      mbar_init(&s_free[t], 4);   // one elected arrive per softmax warp of the tile
-      mbar_init(&p_full[t], 4);
-      mbar_init(&pv_done[t], 1);
-      mbar_init(&mma_done[t], 1);
+      mbar_init(sm.s_full(t), 1);
+      mbar_init(sm.s_free(t), 4);  // one elected arrive per softmax warp of the tile
+      mbar_init(sm.p_full(t), 4);
+      mbar_init(sm.pv_done(t), 1);
+      mbar_init(sm.o_free(t), 4);
+      mbar_init(sm.mma_done(t), 1);
     }
-    *abort_flag = 0;
+    *sm.abort_flag() = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(sm.tmem_slot(), 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = *sm.tmem_slot();
   // Each role runs to its own end; the teardown barrier (id 1, every thread of the CTA) is reached from
   // both sides.
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(PF_CTRL_REGS));
-    prefill_control<D, MODE>(tmQ, tmK, tmV, p, smem, tmem, warp, lane, r0, h, bh, seq_start, n_t, n_kv);
+    prefill_control<D, MODE>(tmQ, tmK, tmV, p, smem, tmem, warp, lane);
     tc_fence_before();
     asm volatile("bar.sync 1, %0;" ::"n"(PF_THREADS) : "memory");
     if (warp == 1) {
       tc_fence_after();
       tmem_dealloc(tmem, 512);
     }
+    if (threadIdx.x == 0) {
+      // This CTA takes no more items.  The last CTA of the launch to finish resets the slot's counters.
+      __threadfence();
+      const unsigned int total = gridDim.x * gridDim.y * gridDim.z;
+      if (atomicAdd(&g_pf_sched[p.sched_slot][1], 1u) == total - 1) {
+        __threadfence();
+        atomicExch(&g_pf_sched[p.sched_slot][0], 0u);
+        atomicExch(&g_pf_sched[p.sched_slot][1], 0u);
+      }
+    }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(PF_SM_REGS));
-    prefill_softmax<D, MODE>(p, smem, tmem, warp, lane, r0, L, h, bh, seq_start, causal, n_t);
+    prefill_softmax<D, MODE>(p, smem, tmem, warp, lane);
     tc_fence_before();
     asm volatile("bar.sync 1, %0;" ::"n"(PF_THREADS) : "memory");
   }

@@ -56,14 +56,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same test with a suspend-time hint: a thread whose phase is not complete yet may be suspended until the
+// phase completes (or the hint expires) instead of re-polling, so waiting roles take no issue slots from
+// the warps that compute.
+constexpr uint32_t MBAR_SUSPEND_HINT_NS = 20000;
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(MBAR_SUSPEND_HINT_NS)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Gives up after `lim` nanoseconds (or as soon
 // as *abort is set by another role of the CTA), records ETA_DEV_TIMEOUT, sets *abort and returns false.
 // Never spins forever.  `abort` may be null (then only the time limit ends the wait).
+// SUSPEND selects the suspend-hint test for the re-polls (the default) or plain polling.
+template <bool SUSPEND = true>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, long long lim) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (SUSPEND ? mbar_try_wait_suspend(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if (abort != nullptr && *abort) return false;
     if ((long long)(globaltimer_ns() - t0) > lim) {
       record_status(1 /* ETA_DEV_TIMEOUT */);
@@ -140,6 +158,35 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same two MMAs with compile-time offsets added inside the instruction sequence: A_OFF / B_OFF are in
+// 16-byte units (the descriptors' start-address field; shared addresses stay below 2^18, so the field does
+// not carry) and TA_OFF in TMEM columns.  One base descriptor per operand stays live instead of one per
+// K-step.
+template <uint32_t A_OFF, uint32_t B_OFF>
+__device__ __forceinline__ void mma_ss_off(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "add.s64 da, %1, %5;\n\t"
+      "add.s64 db, %2, %6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(A_OFF), "n"(B_OFF)
+      : "memory");
+}
+template <uint32_t TA_OFF, uint32_t B_OFF>
+__device__ __forceinline__ void mma_ts_off(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 ta;\n\t.reg .b64 db;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "add.u32 ta, %1, %5;\n\t"
+      "add.s64 db, %2, %6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(TA_OFF), "n"(B_OFF)
       : "memory");
 }
 
