@@ -164,9 +164,8 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
     p.S = S;
     p.nblk = (int)nblk;
   }
-  // The work counter may run past n_items by one per CTA: keep it far from 2^32.
-  if (n_items > (long long)INT_MAX) return ETA_ERR_SHAPE;
-  p.n_items = (int)n_items;
+  // The work counter may run past the work count by one per CTA: keep it far from 2^32.
+  if (n_items > (long long)INT_MAX / 2) return ETA_ERR_SHAPE;
   if (mode == eta::MODE_HSTU) {
     if (!std::isfinite(alpha) || !finite_pos(inv_n)) return ETA_ERR_ARG;
     if (o_dtype != ETA_OUT_BF16) return ETA_ERR_ARG;
@@ -177,7 +176,18 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   if (rc != ETA_OK) return rc;
   int sms = 0;
   if ((rc = sm_count(&sms)) != ETA_OK) return rc;
-  const dim3 grid((unsigned)std::min<long long>(n_items, sms), 1, 1);  // persistent: at most one CTA per SM
+  const long long G = std::min<long long>(n_items, sms);
+  const dim3 grid((unsigned)G, 1, 1);  // persistent: at most one CTA per SM
+  // Dense non-causal items all cost the same.  When their count leaves a last wave at most half full, those
+  // last items are split in two (one Q tile each, keys halved between the CTA's two softmax warpgroups), so
+  // the last wave takes about half an item's time.  Needs at least two key tiles (N > 128).
+  long long n_whole = n_items;
+  if (mode == eta::MODE_DENSE && causal == 0 && N > 128 && n_items > G) {
+    const long long R = n_items % G;
+    if (R > 0 && 2 * R <= G) n_whole = n_items - R;
+  }
+  p.n_whole = (int)n_whole;
+  p.n_items = (int)(n_whole + 2 * (n_items - n_whole));
   p.sched_slot = next_sched_slot();
   p.o = o;
   p.lse = (mode == eta::MODE_HSTU) ? nullptr : lse;

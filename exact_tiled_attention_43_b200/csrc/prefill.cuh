@@ -17,6 +17,10 @@
 // mask); only the diagonal tile and a ragged last tile evaluate a per-element mask.  The grid is persistent
 // (at most one CTA per SM): CTAs take items heaviest-first from a device counter and keep their pipeline
 // running across items, so the next item's Q, K/V and first QK^T overlap the current item's epilogue.
+// Non-causal dense launches whose item count leaves a last wave at most half full turn those last items
+// into split items: one 128-row Q tile whose key range is halved between the two softmax warpgroups, the
+// halves merged inside the CTA (exact: the same rescale identity as the online softmax), so the last wave
+// takes about half an item's time.
 //
 // Roles (12 warps):
 //   warp 0      work fetcher + TMA producer: publishes each item to the other roles through a 2-deep ring,
@@ -83,7 +87,8 @@ struct PrefillParams {
   int H, N, max_len;       // N: dense sequence length
   int BH, S;               // dense: B*H; packed: number of sequences
   int nblk;                // 256-row blocks per (batch|sequence, head)
-  int n_items;             // dense: nblk * BH; packed: nblk * S * H
+  int n_items;             // work indices: n_whole whole items, then two split halves per remaining item
+  int n_whole;             // items (in heaviest-first order) processed whole; the rest are split
   int sched_slot;
   int causal, o_f32;
   float scale_log2;        // softmax: scale * log2(e)
@@ -95,10 +100,29 @@ struct PrefillParams {
 // One work item as the producer publishes it to the other roles.
 struct PfItem {
   int bh, h, seq_start, L;  // dense: bh; packed: head and first packed row of the sequence; rows L
-  int r0;                   // first query row of the item (tile t starts at r0 + 128 t)
-  int n0, n1;               // key tiles seen by Q tile 0 / 1
+  int r0;                   // first query row of the item (whole: tile t starts at r0 + 128 t)
+  int n0, n1;               // whole: key tiles seen by Q tile 0 / 1; split: key tiles [0,n0) / [n0,n0+n1)
+  int split;                // one Q tile at r0, its keys halved between the two softmax warpgroups
   int stop;                 // no more work
 };
+
+// Item-local position of a K (v = 0) or V (v = 1) tile load in the K/V ring.  Whole items load K_0, V_0,
+// K_1, V_1, ... (each shared by both Q tiles).  Split items load, per step j, K_j, K_{n0+j}, V_j, V_{n0+j}
+// (the second warpgroup's pair only while j < n1).
+__device__ __forceinline__ int kv_pos(const PfItem &it, int t, int j, int v) {
+  if (!it.split) return 2 * j + v;
+  const int g = 2 * j + 2 * min(j, it.n1);
+  return g + (v ? (j < it.n1 ? 2 : 1) : 0) + t;
+}
+// Loads of the item in the ring.
+__device__ __forceinline__ int kv_loads(const PfItem &it) {
+  return it.split ? 2 * (it.n0 + it.n1) : 2 * max(it.n0, it.n1);
+}
+// Whether ring position `pos` of the item is read by Q tile (warpgroup) t.
+__device__ __forceinline__ bool kv_owned(const PfItem &it, int t, int pos) {
+  if (!it.split) return pos < 2 * (t ? it.n1 : it.n0);
+  return pos < 4 * it.n1 ? ((pos & 1) == t) : (t == 0);
+}
 
 template <int D>
 struct PfCfg {
@@ -114,8 +138,8 @@ struct PfCfg {
   // barriers: full/empty per stage; q_full, q_empty; item_full[2], item_empty[2];
   // per tile {s_full, s_free, p_full, pv_done, o_free, mma_done}
   static constexpr int NBAR = 2 * NST + 2 + 4 + 2 * 6;
-  static constexpr int SMEM_BYTES =
-      1024 /*alignment slack*/ + (2 + NST) * TILE_BYTES + NBAR * 8 + 2 * (int)sizeof(PfItem) + 16;
+  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + (2 + NST) * TILE_BYTES + NBAR * 8 +
+                                    2 * (int)sizeof(PfItem) + PF_BM * 8 /*split merge*/ + 16;
   static constexpr uint32_t TM_O = 256;                  // O_t at TM_O + D*t
   static constexpr uint32_t TM_P = 384;                  // P_t at TM_P + 64*t (D = 64); S_t's columns [0,64) (D = 128)
 };
@@ -133,7 +157,8 @@ struct PfSmem {
                        B_O_FREE = B_PV_DONE + 2, B_MMA_DONE = B_O_FREE + 2, B_END = B_MMA_DONE + 2;
   static_assert(B_END == C::NBAR, "barrier count");
   static constexpr int OFF_ITEMS = OFF_BAR + C::NBAR * 8;
-  static constexpr int OFF_TMEM_SLOT = OFF_ITEMS + 2 * (int)sizeof(PfItem);
+  static constexpr int OFF_XCH = OFF_ITEMS + 2 * (int)sizeof(PfItem);
+  static constexpr int OFF_TMEM_SLOT = OFF_XCH + PF_BM * 8;
   static constexpr int OFF_ABORT = OFF_TMEM_SLOT + 4;
   uint8_t *base;
   __device__ explicit PfSmem(uint8_t *smem) : base(smem) {}
@@ -158,6 +183,8 @@ struct PfSmem {
   __device__ __forceinline__ uint64_t *o_free(int t) const { return bar(B_O_FREE + t); }
   __device__ __forceinline__ uint64_t *mma_done(int t) const { return bar(B_MMA_DONE + t); }
   __device__ __forceinline__ PfItem *items() const { return reinterpret_cast<PfItem *>(base + OFF_ITEMS); }
+  // split items: (running max, exp-sum) of each query row of the second warpgroup's key half
+  __device__ __forceinline__ float2 *xch() const { return reinterpret_cast<float2 *>(base + OFF_XCH); }
   __device__ __forceinline__ uint32_t *tmem_slot() const { return reinterpret_cast<uint32_t *>(base + OFF_TMEM_SLOT); }
   __device__ __forceinline__ volatile int *abort_flag() const {
     return reinterpret_cast<volatile int *>(base + OFF_ABORT);
@@ -168,6 +195,11 @@ struct PfSmem {
 template <int MODE>
 __device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int idx) {
   PfItem it{};
+  int half = -1;
+  if (idx >= p.n_whole) {  // split halves (only dense non-causal launches with N > 128 have any)
+    half = (idx - p.n_whole) & 1;
+    idx = p.n_whole + ((idx - p.n_whole) >> 1);
+  }
   int blk;
   if constexpr (MODE != MODE_DENSE) {
     const int per = p.S * p.H;
@@ -193,7 +225,15 @@ __device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int idx) {
   const int e1 = (qs1 >= it.L) ? 0 : (causal ? min(it.L, qs1 + PF_BM) : it.L);
   it.n0 = (e0 + PF_BN - 1) / PF_BN;
   it.n1 = (e1 + PF_BN - 1) / PF_BN;
+  it.split = 0;
   it.stop = 0;
+  if (half >= 0) {
+    const int n = (it.L + PF_BN - 1) / PF_BN;  // >= 2
+    it.split = 1;
+    it.r0 += half * PF_BM;
+    it.n0 = (n + 1) / 2;
+    it.n1 = n - it.n0;
+  }
   return it;
 }
 
@@ -238,35 +278,45 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
           if (!ok) break;
         }
         mbar_arrive_expect_tx(sm.q_full(), 2 * C::TILE_BYTES);
+        // Q tile t: rows r0 + 128 t (whole item), or the item's one Q tile in both slots (split item).
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
+          const int qrow = it.r0 + (it.split ? 0 : t * PF_BM);
 #pragma unroll
           for (int c = 0; c < C::KCH; ++c) {
             uint8_t *dst = sm.sQ() + t * C::TILE_BYTES + c * C::CHUNK_BYTES;
             if constexpr (PACKED)
-              tma_load_3d(dst, &tmQ, sm.q_full(), 64 * c, it.h, it.seq_start + it.r0 + t * PF_BM);
+              tma_load_3d(dst, &tmQ, sm.q_full(), 64 * c, it.h, it.seq_start + qrow);
             else
-              tma_load_3d(dst, &tmQ, sm.q_full(), 64 * c, it.r0 + t * PF_BM, it.bh);
+              tma_load_3d(dst, &tmQ, sm.q_full(), 64 * c, qrow, it.bh);
           }
         }
         ++q_issued;
-        const int n_loads = 2 * max(it.n0, it.n1);
-        for (int i = 0; i < n_loads; ++i) {
+        // K/V tiles in ring order (the order kv_pos numbers them).
+        auto load_kv = [&](const CUtensorMap *m, int jt) {
           const int st = kv_issued % C::NST;
-          ok = mbar_wait(sm.empty(st), ((kv_issued / C::NST) & 1) ^ 1, sm.abort_flag(), p.wait_ns);
-          if (!ok) break;
-          const int j = i >> 1;
-          const CUtensorMap *m = (i & 1) ? &tmV : &tmK;
+          if (!mbar_wait(sm.empty(st), ((kv_issued / C::NST) & 1) ^ 1, sm.abort_flag(), p.wait_ns)) return false;
           mbar_arrive_expect_tx(sm.full(st), C::TILE_BYTES);
 #pragma unroll
           for (int c = 0; c < C::KCH; ++c) {
             uint8_t *dst = sm.sKV() + st * C::TILE_BYTES + c * C::CHUNK_BYTES;
             if constexpr (PACKED)
-              tma_load_3d(dst, m, sm.full(st), 64 * c, it.h, it.seq_start + j * PF_BN);
+              tma_load_3d(dst, m, sm.full(st), 64 * c, it.h, it.seq_start + jt * PF_BN);
             else
-              tma_load_3d(dst, m, sm.full(st), 64 * c, j * PF_BN, it.bh);
+              tma_load_3d(dst, m, sm.full(st), 64 * c, jt * PF_BN, it.bh);
           }
           ++kv_issued;
+          return true;
+        };
+        if (!it.split) {
+          const int n_kv = max(it.n0, it.n1);
+          for (int j = 0; ok && j < n_kv; ++j) ok = load_kv(&tmK, j) && load_kv(&tmV, j);
+        } else {
+          for (int j = 0; ok && j < it.n0; ++j) {
+            const bool both = j < it.n1;
+            ok = load_kv(&tmK, j) && (!both || load_kv(&tmK, it.n0 + j)) && load_kv(&tmV, j) &&
+                 (!both || load_kv(&tmV, it.n0 + j));
+          }
         }
       }
       if (!ok) {
@@ -321,11 +371,9 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
         mbar_arrive(sm.item_empty(k & 1));
         if (it.stop) break;
         const int n_t[2] = {it.n0, it.n1};
-        const int n_kv = max(it.n0, it.n1);  // >= 1: an item has at least one row
         ok = mbar_wait(sm.q_full(), k & 1, sm.abort_flag(), p.wait_ns);
         if (!ok) break;
-        // K/V ring: K_j is item-local load 2j, V_j is 2j + 1.
-        auto kv_wait = [&](int i) {
+        auto kv_wait = [&](int i) {  // item-local ring position i (numbered by kv_pos)
           const int g = kv_base + i;
           return mbar_wait(sm.full(g % C::NST), (g / C::NST) & 1, sm.abort_flag(), p.wait_ns);
         };
@@ -339,90 +387,196 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
           // ---------------- issuer 1+t serves Q tile t; the next S_t as soon as S_t is free
           const int t = warp - 1;
           const int nt = (t == 0) ? it.n0 : it.n1;
-          if (nt > 0) {
-            ok = kv_wait(0) && (gs[0] == 0 || mbar_wait(sm.s_free(t), (gs[0] - 1) & 1, sm.abort_flag(), p.wait_ns));
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(t, kv_stage(0));
-            mma_commit(sm.s_full(t));
-            mma_commit(sm.empty(kv_stage(0)));
-            ++gs[0];
-          }
-          if (nt <= 1) mma_commit(sm.q_empty());  // every QK^T of this item is issued
-          for (int j = 0; ok && j < nt; ++j) {
-            if (j + 1 < nt) {
-              ok = kv_wait(2 * j + 2) && mbar_wait(sm.s_free(t), (gs[0] - 1) & 1, sm.abort_flag(), p.wait_ns);
+          if (MODE != MODE_DENSE || !it.split) {
+            const int n_kv = max(it.n0, it.n1);
+            if (nt > 0) {
+              ok = kv_wait(0) && (gs[0] == 0 || mbar_wait(sm.s_free(t), (gs[0] - 1) & 1, sm.abort_flag(), p.wait_ns));
               if (!ok) break;
               tc_fence_after();
-              issue_s(t, kv_stage(2 * j + 2));
-              mma_commit(sm.s_full(t));
-              mma_commit(sm.empty(kv_stage(2 * j + 2)));
-              ++gs[0];
-              if (j + 2 == nt) mma_commit(sm.q_empty());
-            }
-            ok = kv_wait(2 * j + 1) && mbar_wait(sm.p_full(t), gp[0] & 1, sm.abort_flag(), p.wait_ns) &&
-                 (j > 0 || o_wait(t, 0));
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(t, kv_stage(2 * j + 1), j > 0);
-            mma_commit(sm.pv_done(t));
-            mma_commit(sm.empty(kv_stage(2 * j + 1)));
-            ++gp[0];
-          }
-          // Key/value tiles of this item that tile t does not see: release them once they landed.
-          for (int i = 2 * nt; ok && i < 2 * n_kv; ++i) {
-            ok = kv_wait(i);
-            if (ok) mbar_arrive(sm.empty(kv_stage(i)));
-          }
-          if (nt > 0) ++go[0];
-        } else {
-          // ---------------- one issuer for both tiles; P aliased into S; issue order PV_t(j), S_t(j+1)
-          ok = kv_wait(0);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int t = 0; t < 2; ++t)
-            if (n_t[t] > 0) {
               issue_s(t, kv_stage(0));
               mma_commit(sm.s_full(t));
-              ++gs[t];
+              mma_commit(sm.empty(kv_stage(0)));
+              ++gs[0];
             }
-          mma_commit(sm.empty(kv_stage(0)));
-          if (n_kv == 1) mma_commit(sm.q_empty());
-          for (int j = 0; ok && j < n_kv; ++j) {
-            ok = kv_wait(2 * j + 1);
-            if (!ok) break;
-            bool k_ready = false;
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              if (!ok || j >= n_t[t]) continue;
-              ok = mbar_wait(sm.p_full(t), gp[t] & 1, sm.abort_flag(), p.wait_ns) && (j > 0 || o_wait(t, t));
+            if (nt <= 1) mma_commit(sm.q_empty());  // every QK^T of this item is issued
+            for (int j = 0; ok && j < nt; ++j) {
+              if (j + 1 < nt) {
+                ok = kv_wait(2 * j + 2) && mbar_wait(sm.s_free(t), (gs[0] - 1) & 1, sm.abort_flag(), p.wait_ns);
+                if (!ok) break;
+                tc_fence_after();
+                issue_s(t, kv_stage(2 * j + 2));
+                mma_commit(sm.s_full(t));
+                mma_commit(sm.empty(kv_stage(2 * j + 2)));
+                ++gs[0];
+                if (j + 2 == nt) mma_commit(sm.q_empty());
+              }
+              ok = kv_wait(2 * j + 1) && mbar_wait(sm.p_full(t), gp[0] & 1, sm.abort_flag(), p.wait_ns) &&
+                   (j > 0 || o_wait(t, 0));
               if (!ok) break;
               tc_fence_after();
               issue_pv(t, kv_stage(2 * j + 1), j > 0);
               mma_commit(sm.pv_done(t));
-              ++gp[t];
-              if (j + 1 < n_t[t]) {
-                if (!k_ready) {
-                  ok = kv_wait(2 * j + 2);
-                  if (!ok) break;
-                  k_ready = true;
-                }
-                issue_s(t, kv_stage(2 * j + 2));
+              mma_commit(sm.empty(kv_stage(2 * j + 1)));
+              ++gp[0];
+            }
+            // Key/value tiles of this item that tile t does not see: release them once they landed.
+            for (int i = 2 * nt; ok && i < 2 * n_kv; ++i) {
+              ok = kv_wait(i);
+              if (ok) mbar_arrive(sm.empty(kv_stage(i)));
+            }
+          } else {
+            // Ring positions this tile does not read are released (arrive on their empty barrier) in order.
+            // Arriving for position r is in the right phase once the producer has issued load r.  Below a
+            // position of its own that this issuer has just seen land, that holds with no further wait (and
+            // the producer never needs a release at or above that position to issue it: a split item's own
+            // positions are at most 4 apart, a whole item's are a prefix).  Past its last own position the
+            // issuer waits for each position before releasing it.
+            int rel = 0;  // positions below rel are accounted for
+            auto release_below = [&](int pos) {
+              for (; rel < pos; ++rel)
+                if (!kv_owned(it, t, rel)) mbar_arrive(sm.empty(kv_stage(rel)));
+            };
+            if (nt > 0) {
+              const int pk = kv_pos(it, t, 0, 0);
+              ok = kv_wait(pk);
+              if (!ok) break;
+              release_below(pk);
+              ok = gs[0] == 0 || mbar_wait(sm.s_free(t), (gs[0] - 1) & 1, sm.abort_flag(), p.wait_ns);
+              if (!ok) break;
+              tc_fence_after();
+              issue_s(t, kv_stage(pk));
+              mma_commit(sm.s_full(t));
+              mma_commit(sm.empty(kv_stage(pk)));
+              ++gs[0];
+            }
+            if (nt <= 1) mma_commit(sm.q_empty());  // every QK^T of this item is issued
+            for (int j = 0; ok && j < nt; ++j) {
+              if (j + 1 < nt) {
+                const int pk = kv_pos(it, t, j + 1, 0);
+                ok = kv_wait(pk);
+                if (!ok) break;
+                release_below(pk);
+                ok = mbar_wait(sm.s_free(t), (gs[0] - 1) & 1, sm.abort_flag(), p.wait_ns);
+                if (!ok) break;
+                tc_fence_after();
+                issue_s(t, kv_stage(pk));
+                mma_commit(sm.s_full(t));
+                mma_commit(sm.empty(kv_stage(pk)));
+                ++gs[0];
+                if (j + 2 == nt) mma_commit(sm.q_empty());
+              }
+              const int pv = kv_pos(it, t, j, 1);
+              ok = kv_wait(pv);
+              if (!ok) break;
+              release_below(pv);
+              ok = mbar_wait(sm.p_full(t), gp[0] & 1, sm.abort_flag(), p.wait_ns) && (j > 0 || o_wait(t, 0));
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv(t, kv_stage(pv), j > 0);
+              mma_commit(sm.pv_done(t));
+              mma_commit(sm.empty(kv_stage(pv)));
+              ++gp[0];
+            }
+            for (const int tot = kv_loads(it); ok && rel < tot; ++rel) {
+              if (kv_owned(it, t, rel)) continue;
+              ok = kv_wait(rel);
+              if (ok) mbar_arrive(sm.empty(kv_stage(rel)));
+            }
+          }
+          if (nt > 0) ++go[0];
+        } else {
+          // ---------------- one issuer for both tiles; P aliased into S; issue order PV_t(j), S_t(j+1).
+          // A whole item's K_j / V_j serve both tiles (released after both); a split item's each serve one.
+          const int n_kv = max(it.n0, it.n1);  // >= 1: an item has at least one row
+          if (MODE != MODE_DENSE || !it.split) {
+            ok = kv_wait(0);
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+              if (n_t[t] > 0) {
+                issue_s(t, kv_stage(0));
                 mma_commit(sm.s_full(t));
                 ++gs[t];
               }
+            mma_commit(sm.empty(kv_stage(0)));
+            if (n_kv == 1) mma_commit(sm.q_empty());
+            for (int j = 0; ok && j < n_kv; ++j) {
+              ok = kv_wait(2 * j + 1);
+              if (!ok) break;
+              bool k_ready = false;
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                if (!ok || j >= n_t[t]) continue;
+                ok = mbar_wait(sm.p_full(t), gp[t] & 1, sm.abort_flag(), p.wait_ns) && (j > 0 || o_wait(t, t));
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(t, kv_stage(2 * j + 1), j > 0);
+                mma_commit(sm.pv_done(t));
+                ++gp[t];
+                if (j + 1 < n_t[t]) {
+                  if (!k_ready) {
+                    ok = kv_wait(2 * j + 2);
+                    if (!ok) break;
+                    k_ready = true;
+                  }
+                  issue_s(t, kv_stage(2 * j + 2));
+                  mma_commit(sm.s_full(t));
+                  ++gs[t];
+                }
+              }
+              if (!ok) break;
+              mma_commit(sm.empty(kv_stage(2 * j + 1)));
+              if (k_ready) mma_commit(sm.empty(kv_stage(2 * j + 2)));
+              if (j + 2 == n_kv) mma_commit(sm.q_empty());
+            }
+          } else {
+            // Split item: every ring position serves one tile (both tiles have key tiles).
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int pk = kv_pos(it, t, 0, 0);
+              ok = ok && kv_wait(pk);
+              if (!ok) break;
+              tc_fence_after();
+              issue_s(t, kv_stage(pk));
+              mma_commit(sm.s_full(t));
+              mma_commit(sm.empty(kv_stage(pk)));
+              ++gs[t];
             }
             if (!ok) break;
-            mma_commit(sm.empty(kv_stage(2 * j + 1)));
-            if (k_ready) mma_commit(sm.empty(kv_stage(2 * j + 2)));
-            if (j + 2 == n_kv) mma_commit(sm.q_empty());
+            if (n_kv == 1) mma_commit(sm.q_empty());
+            for (int j = 0; ok && j < n_kv; ++j) {
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                if (!ok || j >= n_t[t]) continue;
+                const int pv = kv_pos(it, t, j, 1);
+                ok = kv_wait(pv) && mbar_wait(sm.p_full(t), gp[t] & 1, sm.abort_flag(), p.wait_ns) &&
+                     (j > 0 || o_wait(t, t));
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(t, kv_stage(pv), j > 0);
+                mma_commit(sm.pv_done(t));
+                mma_commit(sm.empty(kv_stage(pv)));
+                ++gp[t];
+                if (j + 1 < n_t[t]) {
+                  const int pk = kv_pos(it, t, j + 1, 0);
+                  ok = kv_wait(pk);
+                  if (!ok) break;
+                  issue_s(t, kv_stage(pk));
+                  mma_commit(sm.s_full(t));
+                  mma_commit(sm.empty(kv_stage(pk)));
+                  ++gs[t];
+                }
+              }
+              if (!ok) break;
+              if (j + 2 == n_kv) mma_commit(sm.q_empty());
+            }
           }
 #pragma unroll
           for (int t = 0; t < 2; ++t)
             if (n_t[t] > 0) ++go[t];
         }
-        kv_base += 2 * n_kv;
+        kv_base += kv_loads(it);
       }
       // Every MMA issued by this thread has completed before TMEM is released.
       mma_commit(sm.mma_done(warp - 1));
@@ -462,9 +616,11 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
     if (lane == 0) mbar_arrive(sm.item_empty(k & 1));
     if (it.stop) break;
     const int L = it.L;
-    const int q_start = it.r0 + t * PF_BM;
+    const int q_start = it.r0 + (it.split ? 0 : t * PF_BM);
     const int qpos = q_start + row;
     const int nt = (t == 0) ? it.n0 : it.n1;
+    const int kv_lo = (it.split && t == 1) ? it.n0 : 0;  // first key tile of this warpgroup
+    const size_t orow = PACKED ? ((size_t)(it.seq_start + qpos) * p.H + it.h) : ((size_t)it.bh * p.N + qpos);
     float m_used = -INFINITY, l = 0.f;
     for (int j = 0; j < nt; ++j, ++gj) {
       ok = mbar_wait(sm.s_full(t), gj & 1, sm.abort_flag(), p.wait_ns);
@@ -482,7 +638,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
         __syncwarp();
         if (lane == 0) mbar_arrive(sm.s_free(t));  // S_t may now be overwritten by the next QK^T
       }
-      const int k0 = j * PF_BN;
+      const int k0 = (kv_lo + j) * PF_BN;
       const bool need_mask = (k0 + PF_BN > L) || (causal && k0 + PF_BN - 1 > q_start);
       const int kmax = causal ? min(L - 1, qpos) - k0 : L - 1 - k0;  // last visible key, tile-local
       uint32_t pk[64];
@@ -603,35 +759,73 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     tc_fence_after();
-    const float inv_l = HSTU ? 1.f : ((l > 0.f) ? 1.f / l : 0.f);
+    // Final row statistics; with a split item the first warpgroup merges the two key halves:
+    //   m = max(m0, m1),  l = l0 2^(m0-m) + l1 2^(m1-m),  O = (O_0 2^(m0-m) + O_1 2^(m1-m)) / l.
+    float m_fin = m_used, l_fin = l, a0 = 1.f, a1 = 0.f;
+    bool merge = false;
+    if constexpr (MODE == MODE_DENSE) {
+      if (it.split) {
+        if (t == 1) {
+          // Hand this row's (m, l) to the first warpgroup, which reads O_1 from TMEM and stores the row.
+          sm.xch()[row] = make_float2(m_used, l);
+          tc_fence_before();
+          asm volatile("bar.arrive 2, %0;" ::"n"(2 * 128) : "memory");
+          continue;
+        }
+        asm volatile("bar.sync 2, %0;" ::"n"(2 * 128) : "memory");
+        tc_fence_after();
+        const float2 x = sm.xch()[row];
+        m_fin = fmaxf(m_used, x.x);
+        const float msub = (m_fin == -INFINITY) ? 0.f : m_fin;
+        a0 = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - msub);
+        a1 = (x.x == -INFINITY) ? 0.f : ex2_approx(x.x - msub);
+        l_fin = l * a0 + x.y * a1;
+        merge = true;
+      }
+    }
+    const float inv_l = HSTU ? 1.f : ((l_fin > 0.f) ? 1.f / l_fin : 0.f);
+    const float w0 = a0 * inv_l, w1 = a1 * inv_l;
     const bool valid = qpos < L;
-    const size_t orow = PACKED ? ((size_t)(it.seq_start + qpos) * p.H + it.h) : ((size_t)it.bh * p.N + qpos);
+    const uint32_t tO1 = tmem + lane_addr + C::TM_O + (uint32_t)D;  // O_1 (read here only when merging)
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
-      uint32_t orr[32];
-      ETA_TMEM_LD_X32(tO + 32u * cc, orr);
-      tmem_wait_ld();
+      float ov[32];
+      {
+        uint32_t orr[32];
+        ETA_TMEM_LD_X32(tO + 32u * cc, orr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(orr[i]) * w0;
+      }
+      if (merge) {
+        uint32_t orr[32];
+        ETA_TMEM_LD_X32(tO1 + 32u * cc, orr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = fmaf(__uint_as_float(orr[i]), w1, ov[i]);
+      }
       if (cc == D / 32 - 1) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(sm.o_free(t));  // the next item's first PV may overwrite O_t
+        if (lane == 0) {
+          mbar_arrive(sm.o_free(t));  // the next item's first PV may overwrite O_t
+          if (merge) mbar_arrive(sm.o_free(1));
+        }
       }
       if (valid) {
         if (p.o_f32) {
           float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow * D + 32 * cc);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(orr[4 * i]) * inv_l, __uint_as_float(orr[4 * i + 1]) * inv_l,
-                                 __uint_as_float(orr[4 * i + 2]) * inv_l, __uint_as_float(orr[4 * i + 3]) * inv_l);
+          for (int i = 0; i < 8; ++i) dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
         } else {
           uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + orow * D + 32 * cc);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(orr[8 * i + 0]) * inv_l, __uint_as_float(orr[8 * i + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(orr[8 * i + 2]) * inv_l, __uint_as_float(orr[8 * i + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(orr[8 * i + 4]) * inv_l, __uint_as_float(orr[8 * i + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(orr[8 * i + 6]) * inv_l, __uint_as_float(orr[8 * i + 7]) * inv_l);
+            w.x = pack_bf16x2(ov[8 * i + 0], ov[8 * i + 1]);
+            w.y = pack_bf16x2(ov[8 * i + 2], ov[8 * i + 3]);
+            w.z = pack_bf16x2(ov[8 * i + 4], ov[8 * i + 5]);
+            w.w = pack_bf16x2(ov[8 * i + 6], ov[8 * i + 7]);
             dst[i] = w;
           }
         }
@@ -639,7 +833,8 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
     }
     if (valid) {
       if constexpr (!HSTU) {
-        if (p.lse != nullptr) p.lse[orow] = (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (p.lse != nullptr)
+          p.lse[orow] = (l_fin > 0.f) ? (m_fin + log2f(l_fin)) * 0.69314718055994531f : -INFINITY;
       }
     }
   }

@@ -54,6 +54,7 @@ def test_large_score_magnitudes():
     k = (k.float() * 4).to(torch.bfloat16)
     for causal in (False, True):
         o, lse = eta.attn_fwd(q, k, v, causal=causal)
+        assert eta.status() == 0
         o_ref, lse_ref = oracle.attn(q, k, v, eta.default_scale(64), causal)
         check_o(o, o_ref, "large scores")
         check_lse(lse, lse_ref, "large scores lse")
@@ -109,3 +110,59 @@ def test_prefill_d128_sweep_sampled(N):
         o_ref, lse_ref = oracle.attn(sl(q), sl(k), sl(v), scale, True, rows=rows)
         check_o(sl(o)[:, :, rows], o_ref, f"sweep N={N} h={h}")
         check_lse(sl(lse)[:, :, rows], lse_ref, "sweep lse")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_more_items_than_sms(d, causal):
+    """B*H*blocks well above the SM count: persistent CTAs take several items each (of unequal work when
+    causal), and every output row is compared."""
+    B, H, N = 2, 40, 1000  # 80 heads x 4 blocks = 320 items
+    q, k, v = (t.to(DEV) for t in inputs.dense_qkv(11, B, H, N, d))
+    scale = eta.default_scale(d)
+    o, lse = eta.attn_fwd(q, k, v, causal=causal, scale=scale)
+    assert eta.status() == 0
+    o_ref, lse_ref = oracle.attn(q, k, v, scale, causal)
+    check_o(o, o_ref, f"items>SMs d={d} causal={causal}")
+    check_lse(lse, lse_ref, "items>SMs lse")
+
+
+def test_repeated_launches_on_two_streams():
+    """Hundreds of launches in a row, alternating between two streams, reuse every work-counter slot more
+    than once: each result must be bit-identical to the first (an item's arithmetic does not depend on
+    which CTA runs it)."""
+    q, k, v = (t.to(DEV) for t in inputs.dense_qkv(12, 1, 6, 700, 64))
+    ref, ref_lse = eta.attn_fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    for i in range(600):
+        s = streams[i % 2]
+        with torch.cuda.stream(s):
+            o = torch.empty_like(ref)
+            lse = torch.empty_like(ref_lse)
+            eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse, stream=s)
+            if i % 50 == 0:
+                outs.append((o, lse))
+    torch.cuda.synchronize()
+    assert eta.status() == 0
+    for o, lse in outs:
+        assert torch.equal(o, ref)
+        assert torch.equal(lse, ref_lse)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("shape", [(1, 20, 2000), (1, 160, 200), (2, 74, 1000)])
+def test_split_tail_items(d, shape):
+    """Non-causal launches whose last wave is at most half full split those items: one Q tile each, keys
+    halved between the CTA's two softmax warpgroups and merged in the CTA.  (1,20,2000): 160 items, 12 split
+    into halves of 8 key tiles; (1,160,200): 12 split items of 2 key tiles, the second ragged; (2,74,1000):
+    592 items = 4 full waves, none split.  Every row compared, in fp32 output."""
+    B, H, N = shape
+    q, k, v = (t.to(DEV) for t in inputs.dense_qkv(13, B, H, N, d))
+    scale = eta.default_scale(d)
+    o, lse = eta.attn_fwd(q, k, v, causal=False, scale=scale, out_dtype=torch.float32)
+    assert eta.status() == 0
+    o_ref, lse_ref = oracle.attn(q, k, v, scale, False)
+    check_o(o, o_ref, f"split tail {shape} d={d}")
+    check_lse(lse, lse_ref, "split tail lse")
