@@ -73,8 +73,8 @@ constexpr int PF_LAUNCH_REGS = 168, PF_CTRL_REGS = 56, PF_SM_REGS = 224;
 static_assert(128 * PF_CTRL_REGS + 32 * PF_SM_WARPS * PF_SM_REGS == PF_THREADS * PF_LAUNCH_REGS, "register split");
 constexpr float PF_RESCALE_THRESHOLD = 8.0f;  // log2 units
 // Work counters of the persistent scheduler, one pair per launch in flight, handed out round-robin by the
-// host: [slot][0] = next item, [slot][1] = CTAs finished.  The last CTA of a launch resets its pair to zero
-// for the launch that reuses the slot.
+// host: [slot][0] = next item, [slot][1] = CTAs that took their last item.  The last CTA of a launch to take
+// its last item resets the pair to zero for the launch that reuses the slot.
 constexpr int PF_SCHED_SLOTS = 256;
 __device__ unsigned int g_pf_sched[PF_SCHED_SLOTS][2];
 
@@ -251,6 +251,18 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
+      // Once this CTA takes no more items it counts itself finished; the last CTA of the launch to do so
+      // returns the slot's counters to zero (no CTA touches them after its final fetch).
+      bool retired = false;
+      auto retire = [&]() {
+        retired = true;
+        __threadfence();
+        if (atomicAdd(&g_pf_sched[p.sched_slot][1], 1u) == gridDim.x - 1) {
+          __threadfence();
+          atomicExch(&g_pf_sched[p.sched_slot][0], 0u);
+          atomicExch(&g_pf_sched[p.sched_slot][1], 0u);
+        }
+      };
       int kv_issued = 0;  // K/V ring loads issued, over all items
       int q_issued = 0;   // items whose Q tiles were loaded
       bool ok = true;
@@ -262,6 +274,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
           if (idx >= (unsigned int)p.n_items) {
             it = PfItem{};
             it.stop = 1;
+            retire();
             break;
           }
           it = decode_item<MODE>(p, (int)idx);
@@ -319,6 +332,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
           }
         }
       }
+      if (!retired) retire();  // abandoned before the work ran out
       if (!ok) {
         // Abandoned pipeline: let copies already in flight land before shared memory is released.
         if (q_issued > 0) mbar_wait(sm.q_full(), (q_issued - 1) & 1, nullptr, p.wait_ns);
@@ -891,16 +905,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     if (warp == 1) {
       tc_fence_after();
       tmem_dealloc(tmem, 512);
-    }
-    if (threadIdx.x == 0) {
-      // This CTA takes no more items.  The last CTA of the launch to finish resets the slot's counters.
-      __threadfence();
-      const unsigned int total = gridDim.x * gridDim.y * gridDim.z;
-      if (atomicAdd(&g_pf_sched[p.sched_slot][1], 1u) == total - 1) {
-        __threadfence();
-        atomicExch(&g_pf_sched[p.sched_slot][0], 0u);
-        atomicExch(&g_pf_sched[p.sched_slot][1], 0u);
-      }
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(PF_SM_REGS));
