@@ -441,6 +441,28 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
                                           "frac_of_peak": gbs / peaks["hbm_gbs"], "bytes_per_step": nbytes}
     del q, kc, vc, ws
     torch.cuda.empty_cache()
+
+    # decode over a paged cache with grouped query heads: batch 64, Hq=32 query heads sharing Hkv=8 kv heads,
+    # d=128, 64-row pages in a shuffled pool, lengths U[8192, 32768]
+    B, Hq, Hkv, d, ps = 64, 32, 8, 128, 64
+    lens = inputs.uniform_lengths(inputs.DECODE_PAGED, B, 8192, 32768)
+    q, kp, vp, table, kl = inputs.paged_decode_inputs(inputs.DECODE_PAGED, B, Hq, Hkv, d, ps, lens, spare_pages=0,
+                                                      device=dev)
+    table, kl = table.to(dev), kl.to(dev)
+    ws = torch.empty(eta.attn_decode_paged_workspace_size(B, Hq, table.shape[1], ps, d), dtype=torch.uint8,
+                     device=dev)
+    od = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+    ld = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    ms, _ = timed_steps(lambda: eta.attn_decode_paged(q, kp, vp, table, kl, workspace=ws, out=od, lse=ld), K, W,
+                        flush, stream, ctx)
+    nbytes = (2.0 * Hkv * d * 2 * float(lens.sum()) + q.numel() * 2 + od.numel() * 2 + ld.numel() * 4 +
+              table.numel() * 4)
+    gbs = nbytes * K / (ctx.max(ms) * 1e-3) / 1e9
+    out["decode_paged_gqa_B64_Hq32_Hkv8_d128_page64_L8k-32k"] = {
+        "value": gbs, "unit": "GB/s", "ms_per_step": ms / K, "frac_of_peak": gbs / peaks["hbm_gbs"],
+        "bytes_per_step": nbytes}
+    del q, kp, vp, ws
+    torch.cuda.empty_cache()
     assert eta.status() == 0
     return out
 
@@ -452,6 +474,7 @@ CASES = {
     "prefill_d128_b2": ("dense", dict(B=2, H=32, N=4096, d=128)),
     "hstu_jagged": ("hstu", dict(S=16, H=4, d=64)),
     "decode_b2": ("decode", dict(B=2, H=32, d=128, Lmax=32768)),
+    "decode_paged_b4": ("decode_paged", dict(B=4, Hq=32, Hkv=8, d=128, ps=64)),
 }
 
 
@@ -473,6 +496,12 @@ def run_case(args):
         cu = inputs.cu_seqlens(lens).to(dev)
         q, k, v = inputs.jagged_qkv(inputs.HSTU_JAGGED, int(lens.sum()), s["H"], s["d"], std=0.5, device=dev)
         fns = [lambda: eta.hstu_fwd_jagged(q, k, v, cu, 4096, 0.125, 1.0 / 4096)]
+    elif kind == "decode_paged":
+        lens = inputs.uniform_lengths(inputs.DECODE_PAGED, 64, 8192, 32768)[: s["B"]]
+        q, kp, vp, table, kl = inputs.paged_decode_inputs(inputs.DECODE_PAGED, s["B"], s["Hq"], s["Hkv"], s["d"],
+                                                          s["ps"], lens, spare_pages=0, device=dev)
+        table, kl = table.to(dev), kl.to(dev)
+        fns = [lambda: eta.attn_decode_paged(q, kp, vp, table, kl)]
     else:
         lens = inputs.uniform_lengths(inputs.DECODE, 64, 8192, 32768)[: s["B"]]
         q, kc, vc, kl = inputs.decode_inputs(inputs.DECODE, s["B"], s["H"], s["Lmax"], s["d"], lens, device=dev)

@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libeta.so")
 _lib = None
 
 ETA_OUT_BF16, ETA_OUT_F32 = 0, 1
-ETA_DEV_OK, ETA_DEV_TIMEOUT, ETA_DEV_BAD_KVLEN, ETA_DEV_BAD_CUSEQ = 0, 1, 2, 3
+ETA_DEV_OK, ETA_DEV_TIMEOUT, ETA_DEV_BAD_KVLEN, ETA_DEV_BAD_CUSEQ, ETA_DEV_BAD_PAGE = 0, 1, 2, 3, 4
 
 # name -> (restype, argtypes); mirrors include/eta.h
 _VP, _I, _F, _SZ, _LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_longlong
@@ -34,6 +34,8 @@ SIGNATURES = {
     "attn_decode_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "attn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _SZ, _VP]),
     "attn_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP]),
+    "attn_decode_paged_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "attn_decode_paged": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _VP, _SZ, _VP]),
     "eta_status": (_I, [_VP]),
     "eta_strerror": (ctypes.c_char_p, [_I]),
     "eta_set_wait_timeout_ns": (None, [_LL]),
@@ -191,6 +193,41 @@ def attn_decode(q, kcache, vcache, kv_lens, scale: float | None = None, workspac
     rc = lib().attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kv_lens), _ptr(out), _ptr(lse), B, H, Lmax, d,
                            scale, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     _check(rc, "attn_decode")
+    return out, lse
+
+
+def attn_decode_paged_workspace_size(B: int, Hq: int, max_pages: int, page_size: int, d: int) -> int:
+    return int(lib().attn_decode_paged_workspace_size(B, Hq, max_pages, page_size, d))
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, kv_lens, scale: float | None = None, workspace=None,
+                      out=None, lse=None, stream=None):
+    """Decode step with grouped query heads over a paged cache: q bf16 [B,Hq,d], page pools bf16
+    [num_pages,Hkv,page_size,d], block_table int32 [B,max_pages] and kv_lens int32 [B] (device).
+    Query head hq reads kv head hq // (Hq // Hkv).  Returns (o bf16 [B,Hq,d], lse fp32 [B,Hq])."""
+    torch = _torch()
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_pages, "k_pages", torch.bfloat16, 4)
+    _need(v_pages, "v_pages", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(kv_lens, "kv_lens", torch.int32, 1)
+    num_pages, Hkv, page_size, d = k_pages.shape
+    B, Hq, dq = q.shape
+    max_pages = block_table.shape[1]
+    if v_pages.shape != k_pages.shape or dq != d or block_table.shape[0] != B or kv_lens.shape != (B,):
+        raise ValueError("inconsistent paged decode shapes")
+    need = attn_decode_paged_workspace_size(B, Hq, max_pages, page_size, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    scale = default_scale(d) if scale is None else float(scale)
+    rc = lib().attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(kv_lens), _ptr(out),
+                                 _ptr(lse), B, Hq, Hkv, num_pages, page_size, max_pages, d, scale, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check(rc, "attn_decode_paged")
     return out, lse
 
 

@@ -13,6 +13,7 @@
 
 #include "eta.h"
 #include "decode.cuh"
+#include "decode_paged.cuh"
 #include "prefill.cuh"
 
 namespace {
@@ -228,6 +229,38 @@ size_t decode_ws_bytes(int B, int H, int Lmax, int d) {
   return o_bytes + n * sizeof(float);
 }
 
+// Page pool [num_pages, Hkv, page_size, d] bf16 viewed as a 3-D tensor {d, page_size, num_pages * Hkv}; box =
+// 64 elements (128 B, one swizzle span) x min(page_size, 32) rows x 1.
+int encode_paged_map(CUtensorMap *m, const void *base, int num_pages, int Hkv, int page_size, int d) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return ETA_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)page_size, (cuuint64_t)num_pages * Hkv};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)page_size * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)std::min(page_size, eta::DPG_ROWS), 1}, estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ETA_OK : ETA_ERR_CUDA;
+}
+
+template <int D>
+int launch_decode_paged(const void *k_pages, const void *v_pages, const eta::PagedDecodeParams &p,
+                        const eta::DecodeParams &cp, cudaStream_t st) {
+  CUtensorMap mk, mv;
+  int rc;
+  if ((rc = encode_paged_map(&mk, k_pages, p.num_pages, p.Hkv, p.page_size, D)) != ETA_OK) return rc;
+  if ((rc = encode_paged_map(&mv, v_pages, p.num_pages, p.Hkv, p.page_size, D)) != ETA_OK) return rc;
+  constexpr int smem = 1024 /*alignment slack*/ + 2 * eta::DPG_STAGES * eta::DPG_ROWS * D * 2;
+  auto ks = eta::decode_paged_split_kernel<D>;
+  if (cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return ETA_ERR_CUDA;
+  ks<<<dim3(p.max_splits, p.Hkv, p.B), eta::DPG_THREADS, smem, st>>>(mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return ETA_ERR_CUDA;
+  eta::decode_combine_kernel<D><<<dim3(cp.H, cp.B), D, 0, st>>>(cp);
+  return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
+}
+
+bool valid_page_size(int ps) { return ps == 16 || ps == 32 || ps == 64 || ps == 128 || ps == 256; }
+
 __global__ void selftest_wait_kernel(long long wait_ns) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
@@ -301,6 +334,68 @@ int attn_decode(const void *q, const void *kcache, const void *vcache, const int
   return d == 64 ? launch_decode<64>(p, st) : launch_decode<128>(p, st);
 }
 
+size_t attn_decode_paged_workspace_size(int B, int Hq, int max_pages, int page_size, int d) {
+  if (B <= 0 || Hq <= 0 || max_pages <= 0 || !valid_page_size(page_size) || (d != 64 && d != 128)) return 0;
+  if ((long long)max_pages * page_size > INT_MAX) return 0;
+  return decode_ws_bytes(B, Hq, max_pages * page_size, d);
+}
+
+int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
+                      const int *kv_lens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages, int page_size,
+                      int max_pages, int d, float scale, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!q || !k_pages || !v_pages || !block_table || !kv_lens || !o || !workspace) return ETA_ERR_NULL;
+  if (d != 64 && d != 128) return ETA_ERR_HEAD_DIM;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || num_pages <= 0 || max_pages <= 0 || B > 65535 || Hkv > 65535)
+    return ETA_ERR_SHAPE;
+  if (Hq % Hkv != 0 || Hq / Hkv > eta::DPG_MAX_G) return ETA_ERR_SHAPE;
+  if (!valid_page_size(page_size)) return ETA_ERR_SHAPE;
+  if ((long long)num_pages * Hkv > INT_MAX || (long long)max_pages * page_size > INT_MAX ||
+      (long long)B * max_pages > INT_MAX)
+    return ETA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(workspace))
+    return ETA_ERR_ALIGN;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ETA_ERR_ALIGN;
+  if (!finite_pos(scale)) return ETA_ERR_ARG;
+  const int Lmax = max_pages * page_size;
+  if (workspace_bytes < decode_ws_bytes(B, Hq, Lmax, d)) return ETA_ERR_WORKSPACE;
+  int rc = check_device();
+  if (rc != ETA_OK) return rc;
+  eta::PagedDecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.block_table = block_table;
+  p.kv_lens = kv_lens;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.num_pages = num_pages;
+  p.page_size = page_size;
+  p.max_pages = max_pages;
+  p.Lmax = Lmax;
+  p.chunk = eta::decode_chunk(Lmax);
+  p.max_splits = eta::decode_max_splits(Lmax);
+  const size_t n = (size_t)B * Hq * p.max_splits;
+  p.part_o = static_cast<float *>(workspace);
+  p.part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + ((n * d * sizeof(float) + 255) & ~size_t(255)));
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_ns = g_wait_ns;
+  // the split merge is the contiguous decode's combine step over the Hq query heads
+  eta::DecodeParams cp{};
+  cp.kv_lens = kv_lens;
+  cp.o = static_cast<__nv_bfloat16 *>(o);
+  cp.lse = lse;
+  cp.part_o = p.part_o;
+  cp.part_lse = p.part_lse;
+  cp.B = B;
+  cp.H = Hq;
+  cp.Lmax = Lmax;
+  cp.chunk = p.chunk;
+  cp.max_splits = p.max_splits;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_decode_paged<64>(k_pages, v_pages, p, cp, st)
+                 : launch_decode_paged<128>(k_pages, v_pages, p, cp, st);
+}
+
 int eta_status(void *stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return ETA_ERR_CUDA;
@@ -325,6 +420,7 @@ const char *eta_strerror(int code) {
     case ETA_DEV_TIMEOUT: return "device: a bounded pipeline wait expired";
     case ETA_DEV_BAD_KVLEN: return "device: kv_lens entry outside [0, Lmax]";
     case ETA_DEV_BAD_CUSEQ: return "device: cu_seqlens decreasing or a sequence longer than max_len";
+    case ETA_DEV_BAD_PAGE: return "device: a block_table entry outside [0, num_pages)";
     default: return "unknown code";
   }
 }

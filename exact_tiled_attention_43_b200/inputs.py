@@ -1,7 +1,8 @@
 """Seeded synthetic inputs shared by the CUDA path's tests/benchmark and the oracle.
 
 This module holds no attention arithmetic: it only draws random tensors and lengths and lays them out
-(dense ``[B,H,N,d]``, packed ``[T,H,d]`` + ``cu_seqlens``, decode caches ``[B,H,Lmax,d]``).
+(dense ``[B,H,N,d]``, packed ``[T,H,d]`` + ``cu_seqlens``, decode caches ``[B,H,Lmax,d]``, page pools
+``[num_pages,Hkv,page_size,d]`` + page tables).
 
 Seeds: ``seed = 1000 * config + {0: q, 1: k, 2: v, 3: lengths}``.  Values are iid normal in fp32,
 multiplied by ``std`` and rounded to bf16; lengths are inclusive uniform integer draws.  Tensors are
@@ -13,8 +14,8 @@ from __future__ import annotations
 import torch
 
 # Config ids follow the workload list: 1 tiny check, 2 prefill d=64, 3 prefill d=128 (+ N sweep),
-# 4 HSTU jagged, 5 decode.
-TINY, PREFILL_D64, PREFILL_D128, HSTU_JAGGED, DECODE = 1, 2, 3, 4, 5
+# 4 HSTU jagged, 5 decode, 6 decode over a paged cache with grouped query heads.
+TINY, PREFILL_D64, PREFILL_D128, HSTU_JAGGED, DECODE, DECODE_PAGED = 1, 2, 3, 4, 5, 6
 
 
 def _gen(device, seed: int) -> torch.Generator:
@@ -72,3 +73,40 @@ def decode_inputs(config: int, B: int, H: int, Lmax: int, d: int, lengths, std: 
             kc[b, :, L:] = float("nan")
             vc[b, :, L:] = float("nan")
     return q, kc, vc, lens
+
+
+def paged_decode_inputs(config: int, B: int, Hq: int, Hkv: int, d: int, page_size: int, lengths,
+                        std: float = 1.0, spare_pages: int = 3, device="cpu", poison_tail: bool = False):
+    """Queries ``[B,Hq,d]``, K/V page pools ``[num_pages,Hkv,page_size,d]`` and a page table ``[B,max_pages]``
+    (int32).  Each sequence gets ceil(L/page_size) pages; the pool holds them plus ``spare_pages`` unused
+    ones, and which physical page backs which logical page is a seeded random permutation (seed + 4).
+    Unused table entries are -1.  With ``poison_tail`` every pool row that no sequence reads (the tail of a
+    last page, spare pages) is NaN, so any read past a sequence's end shows up."""
+    base = 1000 * config
+    lens = torch.as_tensor(lengths, dtype=torch.int32).cpu()
+    need = [(int(L) + page_size - 1) // page_size for L in lens]
+    max_pages = max(1, max(need))
+    num_pages = sum(need) + spare_pages
+    q = normal_bf16((B, Hq, d), base + 0, std, device)
+    kp = normal_bf16((num_pages, Hkv, page_size, d), base + 1, std, device)
+    vp = normal_bf16((num_pages, Hkv, page_size, d), base + 2, std, device)
+    perm = torch.randperm(num_pages, generator=_gen("cpu", base + 4))
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    used = torch.zeros(num_pages, dtype=torch.bool)
+    nxt = 0
+    for b in range(B):
+        for i in range(need[b]):
+            pg = int(perm[nxt])
+            nxt += 1
+            table[b, i] = pg
+            used[pg] = True
+    if poison_tail:
+        valid = torch.zeros(num_pages, page_size, dtype=torch.bool)
+        for b in range(B):
+            L = int(lens[b])
+            for i in range(need[b]):
+                valid[int(table[b, i]), : min(page_size, L - i * page_size)] = True
+        mask = (~valid).to(device)[:, None, :, None].expand(num_pages, Hkv, page_size, d)
+        kp[mask] = float("nan")
+        vp[mask] = float("nan")
+    return q, kp, vp, table, lens

@@ -66,6 +66,7 @@ extern "C" {
 #define ETA_DEV_TIMEOUT 1     /* a bounded pipeline wait expired; the kernel abandoned its tile */
 #define ETA_DEV_BAD_KVLEN 2   /* attn_decode: kv_lens[b] < 0 or > Lmax (clamped into range) */
 #define ETA_DEV_BAD_CUSEQ 3   /* varlen/jagged: cu_seqlens decreasing or a sequence longer than max_len */
+#define ETA_DEV_BAD_PAGE 4    /* attn_decode_paged: a block_table entry outside [0, num_pages) (page 0 read) */
 
 /* Output element type selector for attn_fwd / attn_fwd_varlen. */
 #define ETA_OUT_BF16 0
@@ -133,6 +134,43 @@ ETA_API size_t attn_decode_workspace_size(int B, int H, int Lmax, int d);
 ETA_API int attn_decode(const void *q, const void *kcache, const void *vcache, const int *kv_lens, void *o, float *lse,
                 int B, int H, int Lmax, int d, float scale, void *workspace, size_t workspace_bytes,
                 void *stream);
+
+/*
+ * attn_decode_paged_workspace_size -- bytes of device workspace attn_decode_paged needs (split-KV partials of
+ * every query head).  Returns 0 for invalid sizes.
+ */
+ETA_API size_t attn_decode_paged_workspace_size(int B, int Hq, int max_pages, int page_size, int d);
+
+/*
+ * attn_decode_paged -- one decode step with grouped query heads over a paged KV cache.  The decode step of
+ * "AI attention complexity ledger", section "带宽账：decode 阶段的真正瓶颈", with the two cache-side changes
+ * the pages name: key/value heads shared by groups of query heads (the same section's GQA route for
+ * shrinking the KV cache; "FlashAttention (TH)", section "FlashAttention-2": MQA) and a cache held in fixed
+ * pages reached through a page table (the ops-transformer page: KV-cache management, PagedAttention).
+ * For each b and query head hq, with G = Hq / Hkv and kv head g = hq / G:
+ *   s_j = scale * q[b,hq,:] . K_j,  o[b,hq,:] = sum_j softmax(s)_j V_j,  j = 0 .. kv_lens[b]-1,
+ * where row j of sequence b is row (j % page_size) of page block_table[b][j / page_size], kv head g.
+ *   q           : bf16 [B, Hq, d]
+ *   k_pages     : bf16 [num_pages, Hkv, page_size, d]  (page pool; each (page, kv head) is one contiguous
+ *                 page_size x d block); v_pages : same layout
+ *   block_table : int32 [B, max_pages], device; entries for pages 0 .. ceil(kv_lens[b]/page_size)-1 must lie
+ *                 in [0, num_pages) (others are never read); sequences may share pages
+ *   kv_lens     : int32 [B], device, each in [0, max_pages * page_size]; zero gives o = 0, lse = -inf
+ *   o           : bf16 [B, Hq, d];  lse : fp32 [B, Hq] or NULL
+ *   Hq % Hkv == 0 and Hq / Hkv <= 16; page_size in {16, 32, 64, 128, 256}; d in {64, 128};
+ *   num_pages * Hkv, max_pages * page_size and B * max_pages below 2^31.
+ *   workspace   : device buffer of at least attn_decode_paged_workspace_size(B, Hq, max_pages, page_size, d)
+ *                 bytes, 16-byte aligned, owned by the caller, scratch.
+ * Rows past kv_lens[b] inside the last page are never used (whatever they hold).  The cache is split along
+ * the sequence (split-KV) and the splits merged with logsumexp weights, which is exact.
+ * Errors: ETA_ERR_NULL, ETA_ERR_HEAD_DIM, ETA_ERR_SHAPE, ETA_ERR_ALIGN, ETA_ERR_ARG, ETA_ERR_WORKSPACE,
+ * ETA_ERR_DEVICE, ETA_ERR_CUDA; device status ETA_DEV_BAD_KVLEN (length clamped into range) and
+ * ETA_DEV_BAD_PAGE (an out-of-range page number; page 0 is read in its place).
+ */
+ETA_API int attn_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int *block_table,
+                              const int *kv_lens, void *o, float *lse, int B, int Hq, int Hkv, int num_pages,
+                              int page_size, int max_pages, int d, float scale, void *workspace,
+                              size_t workspace_bytes, void *stream);
 
 /*
  * attn_decode_noalloc -- the same decode step as attn_decode, for callers that cannot allocate device memory

@@ -47,6 +47,8 @@ def _load():
         lib.oracle_hstu_jagged.argtypes = [dp, dp, dp, ip, i, i, i, ctypes.c_double, ctypes.c_double, dp]
         lib.oracle_decode.restype = ctypes.c_int64
         lib.oracle_decode.argtypes = [dp, dp, dp, ip, i, i, i, i, ctypes.c_double, dp, dp]
+        lib.oracle_decode_paged.restype = ctypes.c_int64
+        lib.oracle_decode_paged.argtypes = [dp, dp, dp, ip, ip, i, i, i, i, i, i, ctypes.c_double, dp, dp]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -141,4 +143,26 @@ def decode(q, kcache, vcache, kv_lens, scale: float):
     o = np.zeros((B, H, d), np.float64)
     lse = np.zeros((B, H), np.float64)
     _load().oracle_decode(_dp(q), _dp(kc), _dp(vc), _ip(lens), B, H, Lmax, d, float(scale), _dp(o), _dp(lse))
+    return o, lse
+
+
+def decode_paged(q, k_pages, v_pages, block_table, kv_lens, scale: float):
+    """Decode over a paged cache with grouped query heads: q [B,Hq,d], page pools [num_pages,Hkv,page_size,d],
+    block_table [B,max_pages], kv_lens [B].  Returns (o [B,Hq,d], lse [B,Hq])."""
+    q, kp, vp = _f64(q), _f64(k_pages), _f64(v_pages)
+    bt = _i32(block_table)
+    lens = _i32(kv_lens)
+    num_pages, Hkv, page_size, d = kp.shape
+    B, Hq, dq = q.shape
+    max_pages = bt.shape[1]
+    assert dq == d and vp.shape == kp.shape and bt.shape == (B, max_pages) and lens.shape == (B,)
+    assert Hq % Hkv == 0
+    assert int(lens.min(initial=0)) >= 0 and int(lens.max(initial=0)) <= max_pages * page_size
+    for b in range(B):  # the pages a sequence uses must exist
+        used = bt[b, : (int(lens[b]) + page_size - 1) // page_size]
+        assert used.size == 0 or (int(used.min()) >= 0 and int(used.max()) < num_pages)
+    o = np.zeros((B, Hq, d), np.float64)
+    lse = np.zeros((B, Hq), np.float64)
+    _load().oracle_decode_paged(_dp(q), _dp(kp), _dp(vp), _ip(bt), _ip(lens), B, Hq, Hkv, page_size, max_pages, d,
+                                float(scale), _dp(o), _dp(lse))
     return o, lse

@@ -1,6 +1,6 @@
 /*
  * oracle.c -- plain, slow, fp64 CPU oracle for exact attention, HSTU pointwise attention and the
- * single-query decode step.
+ * single-query decode step (contiguous cache, and paged cache with grouped query heads).
  *
  * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the tests, the smoke check and the benchmark's
  * CPU-baseline leg load this library.  It shares no code, header, table or helper with the CUDA
@@ -173,6 +173,40 @@ EXPORT int64_t oracle_decode(const double *q, const double *kc, const double *vc
         const size_t head = (size_t)u * Lmax * d;
         macs += softmax_attention_row(q + (size_t)u * d, kc + head, (size_t)d, vc + head, (size_t)d, kv_lens[b],
                                       d, scale, o + (size_t)u * d, lse + u);
+    }
+    return 2 * macs;
+}
+
+/*
+ * Decode step over a paged cache with grouped query heads ([LEDGER], decode section; the same section names
+ * GQA as a way to shrink the KV cache; "FlashAttention (TH)", section "FlashAttention-2": MQA; the
+ * ops-transformer page: KV-cache management with PagedAttention).  For each (b, hq) with G = Hq / Hkv:
+ * key/value row j (j < kv_lens[b]) of sequence b is row j % page_size of page block_table[b][j / page_size]
+ * for kv head hq / G, in pools k_pages / v_pages [num_pages, Hkv, page_size, d].  The rows are gathered into
+ * a contiguous [L, d] copy and the plain softmax row above is applied.  o is [B,Hq,d], lse is [B,Hq].
+ */
+EXPORT int64_t oracle_decode_paged(const double *q, const double *k_pages, const double *v_pages,
+                                   const int *block_table, const int *kv_lens, int B, int Hq, int Hkv,
+                                   int page_size, int max_pages, int d, double scale, double *o, double *lse)
+{
+    int64_t macs = 0;
+    const int G = Hq / Hkv;
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : macs)
+    for (int64_t u = 0; u < (int64_t)B * Hq; ++u) {
+        const int b = (int)(u / Hq), hq = (int)(u % Hq), g = hq / G;
+        const int L = kv_lens[b];
+        double *kg = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1) * d);
+        double *vg = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1) * d);
+        for (int j = 0; j < L; ++j) {
+            const int page = block_table[(size_t)b * max_pages + j / page_size];
+            const size_t row = (((size_t)page * Hkv + g) * page_size + (size_t)(j % page_size)) * d;
+            memcpy(kg + (size_t)j * d, k_pages + row, sizeof(double) * d);
+            memcpy(vg + (size_t)j * d, v_pages + row, sizeof(double) * d);
+        }
+        macs += softmax_attention_row(q + (size_t)u * d, kg, (size_t)d, vg, (size_t)d, L, d, scale,
+                                      o + (size_t)u * d, lse + u);
+        free(kg);
+        free(vg);
     }
     return 2 * macs;
 }

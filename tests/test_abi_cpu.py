@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_strerror_covers_codes(L):
-    for c in range(-8, 4):
+    for c in range(-8, 5):
         assert eta.strerror(c) != "unknown code"
     assert eta.strerror(12345) == "unknown code"
 
@@ -79,3 +79,28 @@ def test_decode_host_validation(L):
     assert L.attn_decode(A, A, A, A, A, NUL, 64, 32, 32768, 100, 0.088, A, ws, S) == -2
     assert L.attn_decode(A, MIS, A, A, A, NUL, 64, 32, 32768, 128, 0.088, A, ws, S) == -4
     assert L.attn_decode(A, A, A, A, A, NUL, 64, 32, 32768, 128, 0.0, A, ws, S) == -7
+
+
+def test_paged_decode_host_validation(L):
+    # B, Hq, Hkv, num_pages, page_size, max_pages, d
+    ws = eta.attn_decode_paged_workspace_size(64, 32, 512, 64, 128)
+    assert ws > 0 and ws == eta.attn_decode_workspace_size(64, 32, 512 * 64, 128)
+    assert eta.attn_decode_paged_workspace_size(64, 32, 512, 48, 128) == 0  # page size not a power of two >= 16
+    assert eta.attn_decode_paged_workspace_size(64, 32, 512, 64, 96) == 0
+
+    def call(q=A, kp=A, vp=A, bt=A, kl=A, o=A, B=64, Hq=32, Hkv=8, npg=40000, ps=64, mp=512, d=128, sc=0.088,
+             w=A, wsz=ws):
+        return L.attn_decode_paged(q, kp, vp, bt, kl, o, NUL, B, Hq, Hkv, npg, ps, mp, d, sc, w, wsz, S)
+
+    assert call(bt=NUL) == -1
+    assert call(d=80) == -2
+    assert call(Hq=30) == -3          # Hq not a multiple of Hkv
+    assert call(Hq=8 * 17) == -3      # more than 16 query heads per kv head
+    assert call(ps=48) == -3
+    assert call(npg=0) == -3
+    assert call(npg=(1 << 31) // 8) == -3  # num_pages * Hkv beyond 32-bit coordinates
+    assert call(kp=MIS) == -4
+    assert call(sc=float("nan")) == -7
+    assert call(wsz=ws - 1) == -5
+    rc = call()
+    assert rc in (-6, -8)

@@ -370,3 +370,72 @@ def test_decode_empty_cache():
     q, kc, vc, _ = inputs.decode_inputs(inputs.DECODE, 1, 2, 4, 8, [0])
     o, lse = oracle.decode(q, kc, vc, [0], 0.1)
     assert np.all(o == 0.0) and np.all(np.isneginf(lse))
+
+
+# ----------------------------------------------------------------------------------------------
+# decode over a paged cache with grouped query heads
+# ----------------------------------------------------------------------------------------------
+def _scatter_to_pages(kc, page_size, seed):
+    """Cut a contiguous cache [B,Hkv,Lmax,d] into pages scattered over a pool in a seeded random order
+    (the inverse of the oracle's gather, written independently): returns pool [num_pages,Hkv,ps,d] and
+    the page table [B, max_pages]."""
+    B, Hkv, Lmax, d = kc.shape
+    max_pages = (Lmax + page_size - 1) // page_size
+    num_pages = B * max_pages + 2
+    order = np.random.default_rng(seed).permutation(num_pages)
+    pool = np.full((num_pages, Hkv, page_size, d), np.nan)
+    table = np.zeros((B, max_pages), np.int32)
+    for b in range(B):
+        for i in range(max_pages):
+            phys = int(order[b * max_pages + i])
+            table[b, i] = phys
+            rows = kc[b, :, i * page_size:(i + 1) * page_size]
+            pool[phys, :, :rows.shape[1]] = rows
+    return pool, table
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (6, 1)])
+@pytest.mark.parametrize("page_size", [16, 64])
+def test_paged_decode_equals_contiguous_decode_with_repeated_heads(Hq, Hkv, page_size):
+    # GQA: query head hq reads kv head hq // (Hq/Hkv) -- the same as plain multi-head decode with every kv
+    # head repeated for its group (torch.repeat_interleave).  Paging changes nothing but where rows live.
+    B, Lmax, d = 3, 150, 16
+    lens = [150, 33, 1]
+    _, kc, vc, lens_t = inputs.decode_inputs(inputs.DECODE_PAGED, B, Hkv, Lmax, d, lens, poison_tail=True)
+    q = inputs.normal_bf16((B, Hq, d), 6001)
+    kp, table = _scatter_to_pages(kc.double().numpy(), page_size, 1)
+    vp, table_v = _scatter_to_pages(vc.double().numpy(), page_size, 1)
+    assert np.array_equal(table, table_v)
+    o, lse = oracle.decode_paged(q, kp, vp, table, lens_t, 0.25)
+    G = Hq // Hkv
+    o_ref, lse_ref = oracle.decode(q, kc.repeat_interleave(G, dim=1), vc.repeat_interleave(G, dim=1), lens_t, 0.25)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    np.testing.assert_allclose(o, o_ref, atol=1e-13)
+    np.testing.assert_allclose(lse, lse_ref, atol=1e-13)
+
+
+def test_paged_decode_page_permutation_and_single_token():
+    B, Hq, Hkv, d, ps = 2, 4, 2, 8, 16
+    q, kp, vp, table, lens = inputs.paged_decode_inputs(inputs.DECODE_PAGED, B, Hq, Hkv, d, ps, [37, 1])
+    o, lse = oracle.decode_paged(q, kp, vp, table, lens, 0.5)
+    # relabelling the physical pages (and the table with them) changes nothing
+    perm = np.random.default_rng(3).permutation(kp.shape[0])
+    inv = np.argsort(perm)
+    kp2, vp2 = kp[torch.as_tensor(perm)], vp[torch.as_tensor(perm)]
+    table2 = np.where(table.numpy() >= 0, inv[np.maximum(table.numpy(), 0)], -1).astype(np.int32)
+    o2, lse2 = oracle.decode_paged(q, kp2, vp2, table2, lens, 0.5)
+    np.testing.assert_array_equal(o, o2)
+    np.testing.assert_array_equal(lse, lse2)
+    # one cached token: o is that token's value row for the query head's kv head; lse its scaled score
+    pg = int(table[1, 0])
+    for hq in range(Hq):
+        g = hq // (Hq // Hkv)
+        np.testing.assert_array_equal(o[1, hq], vp[pg, g, 0].double().numpy())
+        s = 0.5 * float((q[1, hq].double() * kp[pg, g, 0].double()).sum())
+        assert abs(lse[1, hq] - s) < 1e-12
+
+
+def test_paged_decode_empty_sequence():
+    q, kp, vp, table, lens = inputs.paged_decode_inputs(inputs.DECODE_PAGED, 2, 2, 1, 8, 16, [0, 5])
+    o, lse = oracle.decode_paged(q, kp, vp, table, lens, 0.1)
+    assert np.all(o[0] == 0.0) and np.all(np.isneginf(lse[0])) and np.all(np.isfinite(lse[1]))
