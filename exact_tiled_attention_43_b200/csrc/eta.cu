@@ -79,10 +79,10 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-// bf16 rows of `d` elements; box = 64 elements (128 B, one swizzle span) x 128 rows.
-// dense  : tensor [BH][N][d]      -> dims {d, N, BH},  box {64, 128, 1}
-// packed : tensor [T][H][d]       -> dims {d, H, T},   box {64, 1, 128}
-int encode_map(CUtensorMap *m, const void *base, bool packed, long long n1, long long n2, int d) {
+// bf16 rows of `d` elements; box = 64 elements (128 B, one swizzle span) x `rows` rows.
+// dense  : tensor [BH][N][d]      -> dims {d, N, BH},  box {64, rows, 1}
+// packed : tensor [T][H][d]       -> dims {d, H, T},   box {64, 1, rows}
+int encode_map(CUtensorMap *m, const void *base, bool packed, long long n1, long long n2, int d, int rows) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return ETA_ERR_CUDA;
   cuuint64_t dims[3], strides[2];
@@ -93,13 +93,13 @@ int encode_map(CUtensorMap *m, const void *base, bool packed, long long n1, long
     dims[2] = (cuuint64_t)n2;
     strides[0] = (cuuint64_t)d * 2;
     strides[1] = (cuuint64_t)n1 * d * 2;
-    box[0] = 64; box[1] = 1; box[2] = 128;
+    box[0] = 64; box[1] = 1; box[2] = (cuuint32_t)rows;
   } else {       // n1 = N, n2 = BH
     dims[1] = (cuuint64_t)n1;
     dims[2] = (cuuint64_t)n2;
     strides[0] = (cuuint64_t)d * 2;
     strides[1] = (cuuint64_t)n1 * d * 2;
-    box[0] = 64; box[1] = 128; box[2] = 1;
+    box[0] = 64; box[1] = (cuuint32_t)rows; box[2] = 1;
   }
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -112,9 +112,10 @@ int launch_prefill(const void *q, const void *k, const void *v, bool packed, lon
                    const eta::PrefillParams &p, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   int rc;
-  if ((rc = encode_map(&mq, q, packed, n1, n2, D)) != ETA_OK) return rc;
-  if ((rc = encode_map(&mk, k, packed, n1, n2, D)) != ETA_OK) return rc;
-  if ((rc = encode_map(&mv, v, packed, n1, n2, D)) != ETA_OK) return rc;
+  // Q tiles are 128 rows; K/V tiles are BN rows.
+  if ((rc = encode_map(&mq, q, packed, n1, n2, D, eta::PF_BM)) != ETA_OK) return rc;
+  if ((rc = encode_map(&mk, k, packed, n1, n2, D, eta::PfCfg<D>::BN)) != ETA_OK) return rc;
+  if ((rc = encode_map(&mv, v, packed, n1, n2, D, eta::PfCfg<D>::BN)) != ETA_OK) return rc;
   auto kern = eta::prefill_kernel<D, MODE>;
   constexpr int smem = eta::PfCfg<D>::SMEM_BYTES;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)

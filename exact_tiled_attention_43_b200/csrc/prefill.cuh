@@ -62,7 +62,6 @@ __device__ __forceinline__ void eta_static_for(F &&f) {
 }
 
 constexpr int PF_BM = 128;            // query rows per Q tile (= TMEM lanes)
-constexpr int PF_BN = 128;            // keys per K/V tile
 constexpr int PF_SM_WARPS = 8;        // softmax warps: 2 Q tiles x 4 lane quarters (one thread per query row)
 constexpr int PF_THREADS = 32 * (4 + PF_SM_WARPS);  // + control warpgroup: TMA, 2 MMA issuers, 1 spare
 // Register split (setmaxnreg): the CTA launches with PF_LAUNCH_REGS per thread; the control warpgroup drops
@@ -126,22 +125,32 @@ __device__ __forceinline__ bool kv_owned(const PfItem &it, int t, int pos) {
 
 template <int D>
 struct PfCfg {
-  static constexpr bool ALIAS_P = (D == 128);
+  // Keys per K/V tile.  (At d = 128, 64-key tiles would leave TMEM room for a separate P -- 2 S + 2 O + 2 P =
+  // 128 + 256 + 64 columns -- so that the next QK^T need not follow the PV that reads P; measured, the
+  // halved tiles cost more in per-tile overhead and MMA latency than that saves: 11 % slower.)
+  static constexpr int BN = 128;
+  // P overwrites S's first columns only when S, O and P of both tiles do not fit in 512 TMEM columns.
+  static constexpr bool ALIAS_P = (2 * BN + 2 * D + BN) > 512;
   static constexpr int N_ISSUERS = ALIAS_P ? 1 : 2;
   static constexpr int KCH = D / 64;                     // 128-byte column chunks per row
-  static constexpr int CHUNK_BYTES = PF_BM * 128;        // 128 rows x 128 B
-  static constexpr int TILE_BYTES = KCH * CHUNK_BYTES;   // one 128 x D bf16 tile
-  static constexpr int NST = (D == 64) ? 8 : 4;          // K/V ring depth (each stage holds one tile)
+  static constexpr int Q_CHUNK = PF_BM * 128;            // 128 rows x 128 B
+  static constexpr int Q_TILE = KCH * Q_CHUNK;           // one 128 x D bf16 Q tile
+  static constexpr int KV_CHUNK = BN * 128;              // BN rows x 128 B
+  static constexpr int KV_TILE = KCH * KV_CHUNK;         // one BN x D bf16 K or V tile
+  static constexpr int NST = (KV_TILE <= 16384) ? 8 : 4;  // K/V ring depth (each stage holds one tile)
   // Of every 8 exp2 pairs, how many use the FMA-pipe polynomial instead of the MUFU.  Off: measured inside
   // this kernel it costs more (issue slots, dependency chains) than the MUFU time it saves.
   static constexpr int POLY_PAIRS = 0;
   // barriers: full/empty per stage; q_full, q_empty; item_full[2], item_empty[2];
   // per tile {s_full, s_free, p_full, pv_done, o_free, mma_done}
   static constexpr int NBAR = 2 * NST + 2 + 4 + 2 * 6;
-  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + (2 + NST) * TILE_BYTES + NBAR * 8 +
+  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + 2 * Q_TILE + NST * KV_TILE + NBAR * 8 +
                                     2 * (int)sizeof(PfItem) + PF_BM * 8 /*split merge*/ + 16;
-  static constexpr uint32_t TM_O = 256;                  // O_t at TM_O + D*t
-  static constexpr uint32_t TM_P = 384;                  // P_t at TM_P + 64*t (D = 64); S_t's columns [0,64) (D = 128)
+  // TMEM columns: S_t at BN*t, O_t at TM_O + D*t, P_t at TM_P + (BN/2)*t (or S_t's first columns if ALIAS_P)
+  static constexpr uint32_t TM_O = 2 * BN;
+  static constexpr uint32_t TM_P = 2 * BN + 2 * D;
+  static_assert(TM_P + (ALIAS_P ? 0 : BN) <= 512, "TMEM columns");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 };
 
 // Shared-memory carve-up, common to every role.  Every member is the base address plus a compile-time
@@ -149,8 +158,8 @@ struct PfCfg {
 template <int D>
 struct PfSmem {
   using C = PfCfg<D>;
-  static constexpr int OFF_KV = 2 * C::TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + C::NST * C::TILE_BYTES;
+  static constexpr int OFF_KV = 2 * C::Q_TILE;
+  static constexpr int OFF_BAR = OFF_KV + C::NST * C::KV_TILE;
   static constexpr int B_FULL = 0, B_EMPTY = C::NST, B_QFULL = 2 * C::NST, B_QEMPTY = B_QFULL + 1,
                        B_ITEM_FULL = B_QEMPTY + 1, B_ITEM_EMPTY = B_ITEM_FULL + 2, B_S_FULL = B_ITEM_EMPTY + 2,
                        B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 2,
@@ -192,8 +201,9 @@ struct PfSmem {
 };
 
 // Work item `idx`, heaviest first: the latest row block of every (batch|sequence, head) comes first.
-template <int MODE>
+template <int D, int MODE>
 __device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int idx) {
+  constexpr int BN = PfCfg<D>::BN;
   PfItem it{};
   int half = -1;
   if (idx >= p.n_whole) {  // split halves (only dense non-causal launches with N > 128 have any)
@@ -223,12 +233,12 @@ __device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int idx) {
   const int qs0 = it.r0, qs1 = it.r0 + PF_BM;
   const int e0 = (qs0 >= it.L) ? 0 : (causal ? min(it.L, qs0 + PF_BM) : it.L);
   const int e1 = (qs1 >= it.L) ? 0 : (causal ? min(it.L, qs1 + PF_BM) : it.L);
-  it.n0 = (e0 + PF_BN - 1) / PF_BN;
-  it.n1 = (e1 + PF_BN - 1) / PF_BN;
+  it.n0 = (e0 + BN - 1) / BN;
+  it.n1 = (e1 + BN - 1) / BN;
   it.split = 0;
   it.stop = 0;
   if (half >= 0) {
-    const int n = (it.L + PF_BN - 1) / PF_BN;  // >= 2
+    const int n = (it.L + BN - 1) / BN;  // >= 2
     it.split = 1;
     it.r0 += half * PF_BM;
     it.n0 = (n + 1) / 2;
@@ -277,7 +287,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
             retire();
             break;
           }
-          it = decode_item<MODE>(p, (int)idx);
+          it = decode_item<D, MODE>(p, (int)idx);
           if (it.r0 < it.L) break;  // row blocks past the end of their sequence have no work
         }
         ok = mbar_wait(sm.item_empty(k & 1), ((k >> 1) & 1) ^ 1, sm.abort_flag(), p.wait_ns);
@@ -290,14 +300,14 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
           ok = mbar_wait(sm.q_empty(), (k - 1) & 1, sm.abort_flag(), p.wait_ns);
           if (!ok) break;
         }
-        mbar_arrive_expect_tx(sm.q_full(), 2 * C::TILE_BYTES);
+        mbar_arrive_expect_tx(sm.q_full(), 2 * C::Q_TILE);
         // Q tile t: rows r0 + 128 t (whole item), or the item's one Q tile in both slots (split item).
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           const int qrow = it.r0 + (it.split ? 0 : t * PF_BM);
 #pragma unroll
           for (int c = 0; c < C::KCH; ++c) {
-            uint8_t *dst = sm.sQ() + t * C::TILE_BYTES + c * C::CHUNK_BYTES;
+            uint8_t *dst = sm.sQ() + t * C::Q_TILE + c * C::Q_CHUNK;
             if constexpr (PACKED)
               tma_load_3d(dst, &tmQ, sm.q_full(), 64 * c, it.h, it.seq_start + qrow);
             else
@@ -309,14 +319,14 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
         auto load_kv = [&](const CUtensorMap *m, int jt) {
           const int st = kv_issued % C::NST;
           if (!mbar_wait(sm.empty(st), ((kv_issued / C::NST) & 1) ^ 1, sm.abort_flag(), p.wait_ns)) return false;
-          mbar_arrive_expect_tx(sm.full(st), C::TILE_BYTES);
+          mbar_arrive_expect_tx(sm.full(st), C::KV_TILE);
 #pragma unroll
           for (int c = 0; c < C::KCH; ++c) {
-            uint8_t *dst = sm.sKV() + st * C::TILE_BYTES + c * C::CHUNK_BYTES;
+            uint8_t *dst = sm.sKV() + st * C::KV_TILE + c * C::KV_CHUNK;
             if constexpr (PACKED)
-              tma_load_3d(dst, m, sm.full(st), 64 * c, it.h, it.seq_start + jt * PF_BN);
+              tma_load_3d(dst, m, sm.full(st), 64 * c, it.h, it.seq_start + jt * C::BN);
             else
-              tma_load_3d(dst, m, sm.full(st), 64 * c, jt * PF_BN, it.bh);
+              tma_load_3d(dst, m, sm.full(st), 64 * c, jt * C::BN, it.bh);
           }
           ++kv_issued;
           return true;
@@ -343,29 +353,30 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
   } else if (warp == 1 || (!C::ALIAS_P && warp == 2)) {
     // ================================================================ MMA issuer(s)
     if (lane == 0) {
-      constexpr uint32_t ID_QK = idesc_bf16_f32(PF_BM, PF_BN, false);
+      constexpr uint32_t ID_QK = idesc_bf16_f32(PF_BM, C::BN, false);
       constexpr uint32_t ID_PV = idesc_bf16_f32(PF_BM, D, true);
       const uint32_t sQa = smem_u32(sm.sQ()), sKVa = smem_u32(sm.sKV());
       // S_t = Q_t K^T : K-steps of 16 elements = 32 bytes inside a 128-byte swizzled row.
       const uint64_t dQ = sdesc_sw128(sQa, 16, 1024), dKV = sdesc_sw128(sKVa, 16, 1024);
-      const uint64_t dV = sdesc_sw128(sKVa, C::CHUNK_BYTES, 1024);
+      const uint64_t dV = sdesc_sw128(sKVa, C::KV_CHUNK, 1024);
       auto issue_s = [&](int t, int st) {
-        const uint64_t da = dQ + (uint64_t)((t * C::TILE_BYTES) >> 4);
-        const uint64_t db = dKV + (uint64_t)((st * C::TILE_BYTES) >> 4);
-        const uint32_t dt = tmem + 128u * t;
+        const uint64_t da = dQ + (uint64_t)((t * C::Q_TILE) >> 4);
+        const uint64_t db = dKV + (uint64_t)((st * C::KV_TILE) >> 4);
+        const uint32_t dt = tmem + (uint32_t)(C::BN * t);
         eta_static_for<D / 16>([&](auto kk_c) {
           constexpr int kk = decltype(kk_c)::value;
-          constexpr uint32_t off = ((uint32_t)(kk >> 2) * C::CHUNK_BYTES + (uint32_t)(kk & 3) * 32u) >> 4;
-          mma_ss_off<off, off>(dt, da, db, ID_QK, kk > 0 ? 1u : 0u);
+          constexpr uint32_t a_off = ((uint32_t)(kk >> 2) * C::Q_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
+          constexpr uint32_t b_off = ((uint32_t)(kk >> 2) * C::KV_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
+          mma_ss_off<a_off, b_off>(dt, da, db, ID_QK, kk > 0 ? 1u : 0u);
         });
       };
       // O_t += P_t V : K-steps of 16 keys = 8 TMEM columns of packed bf16 P, 16 rows (2048 B) of V.
       auto issue_pv = [&](int t, int st, bool acc) {
-        const uint32_t tP = C::ALIAS_P ? tmem + 128u * t : tmem + C::TM_P + 64u * t;
-        const uint64_t db = dV + (uint64_t)((st * C::TILE_BYTES) >> 4);
+        const uint32_t tP = C::ALIAS_P ? tmem + (uint32_t)(C::BN * t) : tmem + C::TM_P + (uint32_t)(C::BN / 2 * t);
+        const uint64_t db = dV + (uint64_t)((st * C::KV_TILE) >> 4);
         const uint32_t dt = tmem + C::TM_O + (uint32_t)(D * t);
         const uint32_t acc0 = acc ? 1u : 0u;
-        eta_static_for<PF_BN / 16>([&](auto kk_c) {
+        eta_static_for<C::BN / 16>([&](auto kk_c) {
           constexpr int kk = decltype(kk_c)::value;
           constexpr uint32_t ta_off = 8u * kk, b_off = (2048u * kk) / 16u;
           mma_ts_off<ta_off, b_off>(dt, tP, db, ID_PV, kk > 0 ? 1u : acc0);
@@ -615,9 +626,10 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
   const int quarter = warp & 3;
   const int row = quarter * 32 + lane;
   const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-  const uint32_t tS = tmem + lane_addr + 128u * t;
+  constexpr int BN = C::BN;
+  const uint32_t tS = tmem + lane_addr + (uint32_t)(BN * t);
   const uint32_t tO = tmem + lane_addr + C::TM_O + (uint32_t)(D * t);
-  const uint32_t tP = C::ALIAS_P ? tS : tmem + lane_addr + C::TM_P + 64u * t;
+  const uint32_t tP = C::ALIAS_P ? tS : tmem + lane_addr + C::TM_P + (uint32_t)(BN / 2 * t);
   const bool causal = HSTU ? true : (p.causal != 0);
   int gj = 0;  // key tiles of Q tile t processed, over all items (phases of s_full, p_full, pv_done)
   bool ok = true;
@@ -641,33 +653,31 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[128];
-      ETA_TMEM_LD_X32(tS + 0u, (sr + 0));
-      ETA_TMEM_LD_X32(tS + 32u, (sr + 32));
-      ETA_TMEM_LD_X32(tS + 64u, (sr + 64));
-      ETA_TMEM_LD_X32(tS + 96u, (sr + 96));
+      uint32_t sr[BN];
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) ETA_TMEM_LD_X32(tS + 32u * cc, (sr + 32 * cc));
       tmem_wait_ld();
       if constexpr (!C::ALIAS_P) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(sm.s_free(t));  // S_t may now be overwritten by the next QK^T
       }
-      const int k0 = (kv_lo + j) * PF_BN;
-      const bool need_mask = (k0 + PF_BN > L) || (causal && k0 + PF_BN - 1 > q_start);
+      const int k0 = (kv_lo + j) * BN;
+      const bool need_mask = (k0 + BN > L) || (causal && k0 + BN - 1 > q_start);
       const int kmax = causal ? min(L - 1, qpos) - k0 : L - 1 - k0;  // last visible key, tile-local
-      uint32_t pk[64];
+      uint32_t pk[BN / 2];
       bool resc = false;
       float f = 1.f, rowsum = 0.f, m_new = m_used;
       if constexpr (!HSTU) {
         if (need_mask) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
+          for (int c = 0; c < BN; ++c)
             if (c > kmax) sr[c] = __float_as_uint(-INFINITY);
         }
         // row max: four independent 3-input max chains
         float mxa = -INFINITY, mxb = -INFINITY, mxc = -INFINITY, mxd = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; c += 8) {
+        for (int c = 0; c < BN; c += 8) {
           mxa = max3f(mxa, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
           mxb = max3f(mxb, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
           mxc = max3f(mxc, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
@@ -685,7 +695,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
         // unmasked tiles, the rest (and every element of a masked tile) to the MUFU.
         auto exp_row = [&](auto use_poly) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
+          for (int i = 0; i < BN / 2; ++i) {
             const uint64_t x2 =
                 fma_x2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), cs2, nm2);
             float x0, x1, p0, p1;
@@ -712,7 +722,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
         // HSTU: p = inv_n * silu(alpha s) = h + h * tanh(alpha s / 2),  h = (alpha * inv_n / 2) s
         const uint64_t ha2 = f2pack(p.hstu_half_alpha, p.hstu_half_alpha), ho2 = f2pack(p.hstu_out, p.hstu_out);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < BN / 2; ++i) {
           const int c0 = 2 * i;
           const uint64_t s2 = f2pack(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1]));
           float y0, y1;
@@ -738,8 +748,8 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
           tc_fence_after();
         }
       }
-      ETA_TMEM_ST_X32(tP + 0u, (pk + 0));
-      ETA_TMEM_ST_X32(tP + 32u, (pk + 32));
+#pragma unroll
+      for (int cc = 0; cc < BN / 64; ++cc) ETA_TMEM_ST_X32(tP + 32u * cc, (pk + 32 * cc));
       if constexpr (!HSTU) {
         if (__any_sync(0xffffffffu, resc && j > 0)) {
           const uint64_t f2 = f2pack(f, f);
