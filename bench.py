@@ -425,6 +425,17 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
                                                   "frac_of_peak": tf / pk}
         del q, k, v, o
 
+    # head dim 256 (the FlashAttention-2 head size), B4 H16 N4096 causal: the same H*d as the d=128 line
+    B_, H_, N_ = 4, 16, 4096
+    q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, B_, H_, N_, 256, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B_, H_, N_), dtype=torch.float32, device=dev)
+    ms, _ = timed_steps(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse), K, W, flush, stream, ctx)
+    tf = 2.0 * B_ * H_ * N_ * N_ * 256 * K / (ctx.max(ms) * 1e-3) / 1e12
+    out["prefill_B4_H16_N4096_d256_causal"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+                                               "frac_of_peak": tf / pk}
+    del q, k, v, o, lse
+
     # decode: batch 64, H=32, d=128, lengths U[8192, 32768] (inputs far larger than L2: no flush needed)
     B, H, d, Lmax = 64, 32, 128, 32768
     lens = inputs.uniform_lengths(inputs.DECODE, B, 8192, 32768)
@@ -472,6 +483,7 @@ CASES = {
     "prefill_d64_headline": ("dense", dict(B=1, H=32, N=4096, d=64)),
     "prefill_d64_b4": ("dense", dict(B=4, H=32, N=4096, d=64)),
     "prefill_d128_b2": ("dense", dict(B=2, H=32, N=4096, d=128)),
+    "prefill_d256_b2": ("dense", dict(B=2, H=16, N=4096, d=256)),
     "hstu_jagged": ("hstu", dict(S=16, H=4, d=64)),
     "decode_b2": ("decode", dict(B=2, H=32, d=128, Lmax=32768)),
     "decode_paged_b4": ("decode_paged", dict(B=4, Hq=32, Hkv=8, d=128, ps=64)),

@@ -15,6 +15,7 @@
 #include "decode.cuh"
 #include "decode_paged.cuh"
 #include "prefill.cuh"
+#include "prefill_wide.cuh"
 
 namespace {
 
@@ -107,6 +108,23 @@ int encode_map(CUtensorMap *m, const void *base, bool packed, long long n1, long
   return r == CUDA_SUCCESS ? ETA_OK : ETA_ERR_CUDA;
 }
 
+template <int MODE>
+int launch_prefill_wide(const void *q, const void *k, const void *v, bool packed, long long n1, long long n2,
+                        dim3 grid, const eta::PrefillParams &p, cudaStream_t stream) {
+  constexpr int D = eta::WideCfg::D;
+  CUtensorMap mq, mk, mv;
+  int rc;
+  if ((rc = encode_map(&mq, q, packed, n1, n2, D, eta::PF_BM)) != ETA_OK) return rc;
+  if ((rc = encode_map(&mk, k, packed, n1, n2, D, eta::WideCfg::BN)) != ETA_OK) return rc;
+  if ((rc = encode_map(&mv, v, packed, n1, n2, D, eta::WideCfg::BN)) != ETA_OK) return rc;
+  auto kern = eta::prefill_wide_kernel<MODE>;
+  constexpr int smem = eta::WideCfg::SMEM_BYTES;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ETA_ERR_CUDA;
+  kern<<<grid, eta::WideCfg::THREADS, smem, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
+}
+
 template <int D, int MODE>
 int launch_prefill(const void *q, const void *k, const void *v, bool packed, long long n1, long long n2, dim3 grid,
                    const eta::PrefillParams &p, cudaStream_t stream) {
@@ -135,7 +153,9 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
                    float scale, int causal, int o_dtype, float alpha, float inv_n, void *stream) {
   if (!q || !k || !v || !o) return ETA_ERR_NULL;
   if (mode != eta::MODE_DENSE && !cu_seqlens) return ETA_ERR_NULL;
-  if (d != 64 && d != 128) return ETA_ERR_HEAD_DIM;
+  // head dims 64 and 128 (two 128-row Q tiles per work item); 256 for softmax attention (one Q tile per item)
+  if (d != 64 && d != 128 && !(d == 256 && mode != eta::MODE_HSTU)) return ETA_ERR_HEAD_DIM;
+  const long long rows_per_item = (d == 256) ? eta::PF_BM : 2 * eta::PF_BM;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ETA_ERR_ALIGN;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ETA_ERR_ALIGN;
   if (o_dtype != ETA_OUT_BF16 && o_dtype != ETA_OUT_F32) return ETA_ERR_ARG;
@@ -146,7 +166,7 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   if (mode == eta::MODE_DENSE) {
     if (B <= 0 || N <= 0) return ETA_ERR_SHAPE;
     const long long bh = (long long)B * H;
-    const long long nblk = ((long long)N + 255) / 256;
+    const long long nblk = ((long long)N + rows_per_item - 1) / rows_per_item;
     if (bh > INT_MAX || nblk > 65535) return ETA_ERR_SHAPE;
     n_items = bh * nblk;
     n1 = N;
@@ -157,7 +177,7 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   } else {
     if (S <= 0 || max_len <= 0 || T_total < 0 || S > 65535) return ETA_ERR_SHAPE;
     if (T_total == 0) return ETA_OK;  // nothing to compute
-    const long long nblk = ((long long)max_len + 255) / 256;
+    const long long nblk = ((long long)max_len + rows_per_item - 1) / rows_per_item;
     if (nblk > 65535) return ETA_ERR_SHAPE;
     n_items = (long long)S * H * nblk;
     n1 = H;
@@ -184,7 +204,7 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   // last items are split in two (one Q tile each, keys halved between the CTA's two softmax warpgroups), so
   // the last wave takes about half an item's time.  Needs at least two key tiles (N > 128).
   long long n_whole = n_items;
-  if (mode == eta::MODE_DENSE && causal == 0 && N > 128 && n_items > G) {
+  if (mode == eta::MODE_DENSE && causal == 0 && d <= 128 && N > 128 && n_items > G) {
     const long long R = n_items % G;
     if (R > 0 && 2 * R <= G) n_whole = n_items - R;
   }
@@ -203,6 +223,10 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   p.wait_ns = g_wait_ns;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool packed = (mode != eta::MODE_DENSE);
+  if (d == 256) {
+    if (mode == eta::MODE_DENSE) return launch_prefill_wide<eta::MODE_DENSE>(q, k, v, packed, n1, n2, grid, p, st);
+    return launch_prefill_wide<eta::MODE_VARLEN>(q, k, v, packed, n1, n2, grid, p, st);
+  }
   if (d == 64) {
     if (mode == eta::MODE_DENSE) return launch_prefill<64, eta::MODE_DENSE>(q, k, v, packed, n1, n2, grid, p, st);
     if (mode == eta::MODE_VARLEN) return launch_prefill<64, eta::MODE_VARLEN>(q, k, v, packed, n1, n2, grid, p, st);
@@ -411,7 +435,7 @@ const char *eta_strerror(int code) {
   switch (code) {
     case ETA_OK: return "ok";
     case ETA_ERR_NULL: return "a required pointer is NULL";
-    case ETA_ERR_HEAD_DIM: return "head dimension must be 64 or 128";
+    case ETA_ERR_HEAD_DIM: return "unsupported head dimension (64, 128; 256 for attn_fwd / attn_fwd_varlen)";
     case ETA_ERR_SHAPE: return "a size is out of range or inconsistent";
     case ETA_ERR_ALIGN: return "a tensor pointer is not 16-byte aligned";
     case ETA_ERR_WORKSPACE: return "workspace is smaller than attn_decode_workspace_size()";

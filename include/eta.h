@@ -53,7 +53,7 @@ extern "C" {
 /* Host-side error codes (negative) returned by the entry points. */
 #define ETA_OK 0
 #define ETA_ERR_NULL (-1)      /* a required pointer is NULL */
-#define ETA_ERR_HEAD_DIM (-2)  /* d is not 64 or 128 */
+#define ETA_ERR_HEAD_DIM (-2)  /* d is not 64 or 128 (or 256, for attn_fwd / attn_fwd_varlen) */
 #define ETA_ERR_SHAPE (-3)     /* a size is <= 0, too large for 32-bit indexing, or inconsistent */
 #define ETA_ERR_ALIGN (-4)     /* a tensor pointer is not 16-byte aligned */
 #define ETA_ERR_WORKSPACE (-5) /* workspace smaller than attn_decode_workspace_size() */
@@ -81,6 +81,8 @@ extern "C" {
  *             may be NULL (not written)
  *   scale   : multiplies Q K^T before the softmax (1/sqrt(d) in the formula); finite and > 0
  *   causal  : 0 = every key; 1 = query i sees keys j <= i (top-left aligned, diagonal included)
+ *   d       : 64, 128 or 256 (256 is the FlashAttention-2 head size, "FlashAttention (TH)", section
+ *             "FlashAttention-2"; it runs one 128-row Q tile per work item, see prefill_wide.cuh)
  * Errors: ETA_ERR_NULL, ETA_ERR_HEAD_DIM, ETA_ERR_SHAPE (B,H,N <= 0 or B*H*N*d >= 2^31), ETA_ERR_ALIGN,
  *         ETA_ERR_ARG, ETA_ERR_DEVICE, ETA_ERR_CUDA.
  */

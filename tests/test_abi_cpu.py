@@ -57,6 +57,10 @@ def test_attn_fwd_host_validation(L):
     # valid arguments without a usable GPU: a clean negative code, no crash
     rc = L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 64, 0.125, 0, 0, S)
     assert rc in (-6, -8)
+    # head dim 256: accepted for softmax attention (dense and packed), not for HSTU
+    assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 256, 0.0625, 1, 0, S) in (-6, -8)
+    assert L.attn_fwd_varlen(A, A, A, A, NUL, A, 2, 128, 256, 1, 256, 0.0625, 1, 0, S) in (-6, -8)
+    assert L.hstu_fwd_jagged(A, A, A, A, A, 2, 128, 256, 1, 256, 0.125, 1.0, S) == -2
 
 
 def test_varlen_and_hstu_host_validation(L):
