@@ -436,6 +436,19 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
                                                "frac_of_peak": tf / pk}
     del q, k, v, o, lse
 
+    # e4m3 inputs with per-tensor descales, B8 H32 N4096 d128 causal (the d=128 line's shape); the fraction is
+    # of the e4m3 tensor peak, taken as twice the measured bf16 figure (the nominal dense ratio)
+    q8, k8, v8, (dq, dk, dv) = inputs.fp8_dense_qkv(inputs.PREFILL_FP8, 8, 32, 4096, 128, device=dev)
+    o = torch.empty((8, 32, 4096, 128), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((8, 32, 4096), dtype=torch.float32, device=dev)
+    ms, _ = timed_steps(lambda: eta.attn_fwd_fp8(q8, k8, v8, dq, dk, dv, causal=True, out=o, lse=lse), K, W, flush,
+                        stream, ctx)
+    tf = 2.0 * 8 * 32 * 4096 * 4096 * 128 * K / (ctx.max(ms) * 1e-3) / 1e12
+    out["prefill_fp8_B8_H32_N4096_d128_causal"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+                                                   "frac_of_peak": tf / (2.0 * pk),
+                                                   "peak_note": "e4m3 peak = 2 x measured bf16"}
+    del q8, k8, v8, o, lse
+
     # decode: batch 64, H=32, d=128, lengths U[8192, 32768] (inputs far larger than L2: no flush needed)
     B, H, d, Lmax = 64, 32, 128, 32768
     lens = inputs.uniform_lengths(inputs.DECODE, B, 8192, 32768)

@@ -35,6 +35,7 @@ SIGNATURES = {
     "attn_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _SZ, _VP]),
     "attn_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP]),
     "attn_decode_paged_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "attn_fwd_fp8": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _F, _F, _F, _I, _I, _VP]),
     "attn_decode_paged": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _VP, _SZ, _VP]),
     "eta_status": (_I, [_VP]),
     "eta_strerror": (ctypes.c_char_p, [_I]),
@@ -129,6 +130,31 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out_dtyp
                         int(bool(causal)), odt, _stream_ptr(stream))
     _check(rc, "attn_fwd")
     return out, (lse if return_lse else None)
+
+
+def attn_fwd_fp8(q8, k8, v8, q_descale: float, k_descale: float, v_descale: float, causal: bool = False,
+                 scale: float | None = None, out_dtype=None, out=None, lse=None, return_lse: bool = True,
+                 stream=None):
+    """Exact attention on e4m3 inputs: q8, k8, v8 torch.float8_e4m3fn [B,H,N,128] with per-tensor descale
+    factors (Q = q8 * q_descale, ...).  Returns (o [B,H,N,128] bf16 or fp32, lse fp32 [B,H,N] or None)."""
+    torch = _torch()
+    for t, name in ((q8, "q8"), (k8, "k8"), (v8, "v8")):
+        _need(t, name, torch.float8_e4m3fn, 4)
+    if k8.shape != q8.shape or v8.shape != q8.shape:
+        raise ValueError("q8, k8, v8 must have the same shape")
+    B, H, N, d = q8.shape
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    odt = {torch.bfloat16: 0, torch.float32: 1}[out_dtype]
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=out_dtype, device=q8.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    scale = default_scale(d) if scale is None else float(scale)
+    rc = lib().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(out), _ptr(lse) if lse is not None else None, B, H, N,
+                            d, scale, float(q_descale), float(k_descale), float(v_descale), int(bool(causal)), odt,
+                            _stream_ptr(stream))
+    _check(rc, "attn_fwd_fp8")
+    return out, lse
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens, max_len: int, causal: bool = False, scale: float | None = None,

@@ -83,7 +83,9 @@ EncodeTiledFn get_encode() {
 // bf16 rows of `d` elements; box = 64 elements (128 B, one swizzle span) x `rows` rows.
 // dense  : tensor [BH][N][d]      -> dims {d, N, BH},  box {64, rows, 1}
 // packed : tensor [T][H][d]       -> dims {d, H, T},   box {64, 1, rows}
-int encode_map(CUtensorMap *m, const void *base, bool packed, long long n1, long long n2, int d, int rows) {
+// `elt` bytes per element: 2 (bf16) or 1 (e4m3, mapped as bytes); the box always spans 128 bytes of a row.
+int encode_map(CUtensorMap *m, const void *base, bool packed, long long n1, long long n2, int d, int rows,
+               int elt = 2) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return ETA_ERR_CUDA;
   cuuint64_t dims[3], strides[2];
@@ -92,17 +94,17 @@ int encode_map(CUtensorMap *m, const void *base, bool packed, long long n1, long
   if (packed) {  // n1 = H, n2 = T
     dims[1] = (cuuint64_t)n1;
     dims[2] = (cuuint64_t)n2;
-    strides[0] = (cuuint64_t)d * 2;
-    strides[1] = (cuuint64_t)n1 * d * 2;
-    box[0] = 64; box[1] = 1; box[2] = (cuuint32_t)rows;
+    strides[0] = (cuuint64_t)d * elt;
+    strides[1] = (cuuint64_t)n1 * d * elt;
+    box[0] = (cuuint32_t)(128 / elt); box[1] = 1; box[2] = (cuuint32_t)rows;
   } else {       // n1 = N, n2 = BH
     dims[1] = (cuuint64_t)n1;
     dims[2] = (cuuint64_t)n2;
-    strides[0] = (cuuint64_t)d * 2;
-    strides[1] = (cuuint64_t)n1 * d * 2;
-    box[0] = 64; box[1] = (cuuint32_t)rows; box[2] = 1;
+    strides[0] = (cuuint64_t)d * elt;
+    strides[1] = (cuuint64_t)n1 * d * elt;
+    box[0] = (cuuint32_t)(128 / elt); box[1] = (cuuint32_t)rows; box[2] = 1;
   }
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+  CUresult r = enc(m, (elt == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16), 3, const_cast<void *>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ETA_OK : ETA_ERR_CUDA;
@@ -125,17 +127,18 @@ int launch_prefill_wide(const void *q, const void *k, const void *v, bool packed
   return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool F8 = false>
 int launch_prefill(const void *q, const void *k, const void *v, bool packed, long long n1, long long n2, dim3 grid,
                    const eta::PrefillParams &p, cudaStream_t stream) {
+  using C = eta::PfCfg<D, F8>;
   CUtensorMap mq, mk, mv;
   int rc;
   // Q tiles are 128 rows; K/V tiles are BN rows.
-  if ((rc = encode_map(&mq, q, packed, n1, n2, D, eta::PF_BM)) != ETA_OK) return rc;
-  if ((rc = encode_map(&mk, k, packed, n1, n2, D, eta::PfCfg<D>::BN)) != ETA_OK) return rc;
-  if ((rc = encode_map(&mv, v, packed, n1, n2, D, eta::PfCfg<D>::BN)) != ETA_OK) return rc;
-  auto kern = eta::prefill_kernel<D, MODE>;
-  constexpr int smem = eta::PfCfg<D>::SMEM_BYTES;
+  if ((rc = encode_map(&mq, q, packed, n1, n2, D, eta::PF_BM, C::ELT)) != ETA_OK) return rc;
+  if ((rc = encode_map(&mk, k, packed, n1, n2, D, C::BN, C::ELT)) != ETA_OK) return rc;
+  if ((rc = encode_map(&mv, v, packed, n1, n2, D, C::BN, C::ELT)) != ETA_OK) return rc;
+  auto kern = eta::prefill_kernel<D, MODE, F8>;
+  constexpr int smem = C::SMEM_BYTES;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ETA_ERR_CUDA;
   // The kernel re-splits its registers between warpgroups (setmaxnreg); the split only adds up when the
@@ -150,9 +153,12 @@ bool finite_pos(float x) { return std::isfinite(x) && x > 0.f; }
 
 int prefill_common(int mode, const void *q, const void *k, const void *v, void *o, float *lse,
                    const int *cu_seqlens, int B, int S, int N, int max_len, int T_total, int H, int d,
-                   float scale, int causal, int o_dtype, float alpha, float inv_n, void *stream) {
+                   float scale, int causal, int o_dtype, float alpha, float inv_n, void *stream, bool f8 = false,
+                   float qk_descale = 1.f, float v_descale = 1.f) {
   if (!q || !k || !v || !o) return ETA_ERR_NULL;
   if (mode != eta::MODE_DENSE && !cu_seqlens) return ETA_ERR_NULL;
+  if (f8 && d != 128) return ETA_ERR_HEAD_DIM;  // e4m3: one 128-byte swizzle span per row
+  if (f8 && (!finite_pos(qk_descale) || !finite_pos(v_descale))) return ETA_ERR_ARG;
   // head dims 64 and 128 (two 128-row Q tiles per work item); 256 for softmax attention (one Q tile per item)
   if (d != 64 && d != 128 && !(d == 256 && mode != eta::MODE_HSTU)) return ETA_ERR_HEAD_DIM;
   const long long rows_per_item = (d == 256) ? eta::PF_BM : 2 * eta::PF_BM;
@@ -217,12 +223,14 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   p.H = H;
   p.causal = causal;
   p.o_f32 = (o_dtype == ETA_OUT_F32);
-  p.scale_log2 = scale * 1.4426950408889634f;
+  p.scale_log2 = scale * qk_descale * 1.4426950408889634f;
   p.hstu_half_alpha = 0.5f * alpha;
   p.hstu_out = 0.5f * alpha * inv_n;
+  p.o_scale = v_descale;
   p.wait_ns = g_wait_ns;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool packed = (mode != eta::MODE_DENSE);
+  if (f8) return launch_prefill<128, eta::MODE_DENSE, true>(q, k, v, packed, n1, n2, grid, p, st);
   if (d == 256) {
     if (mode == eta::MODE_DENSE) return launch_prefill_wide<eta::MODE_DENSE>(q, k, v, packed, n1, n2, grid, p, st);
     return launch_prefill_wide<eta::MODE_VARLEN>(q, k, v, packed, n1, n2, grid, p, st);
@@ -312,6 +320,14 @@ int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float 
                     int max_len, int T_total, int H, int d, float scale, int causal, int o_dtype, void *stream) {
   return prefill_common(eta::MODE_VARLEN, q, k, v, o, lse, cu_seqlens, 0, S, 0, max_len, T_total, H, d, scale, causal,
                         o_dtype, 0.f, 1.f, stream);
+}
+
+int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N, int d,
+                 float scale, float q_descale, float k_descale, float v_descale, int causal, int o_dtype,
+                 void *stream) {
+  if (!finite_pos(q_descale) || !finite_pos(k_descale)) return ETA_ERR_ARG;
+  return prefill_common(eta::MODE_DENSE, q, k, v, o, lse, nullptr, B, 0, N, 0, 0, H, d, scale, causal, o_dtype, 0.f,
+                        1.f, stream, true, q_descale * k_descale, v_descale);
 }
 
 int hstu_fwd_jagged(const void *q, const void *k, const void *v, void *o, const int *cu_seqlens, int S, int max_len,

@@ -93,6 +93,7 @@ struct PrefillParams {
   float scale_log2;        // softmax: scale * log2(e)
   float hstu_half_alpha;   // HSTU: 0.5 * alpha      (tanh argument scale)
   float hstu_out;          // HSTU: 0.5 * alpha * inv_n
+  float o_scale;           // multiplies O / l (1; the V descale factor for e4m3 inputs)
   long long wait_ns;
 };
 
@@ -123,20 +124,26 @@ __device__ __forceinline__ bool kv_owned(const PfItem &it, int t, int pos) {
   return pos < 4 * it.n1 ? ((pos & 1) == t) : (t == 0);
 }
 
-template <int D>
+// F8: Q, K, V are e4m3 (one byte per element), P is rounded to e4m3 for the PV MMA (kind::f8f6f4).
+template <int D, bool F8 = false>
 struct PfCfg {
+  static constexpr int ELT = F8 ? 1 : 2;                 // bytes per input element
+  static constexpr int ROW_BYTES = D * ELT;
   // Keys per K/V tile.  (At d = 128, 64-key tiles would leave TMEM room for a separate P -- 2 S + 2 O + 2 P =
   // 128 + 256 + 64 columns -- so that the next QK^T need not follow the PV that reads P; measured, the
   // halved tiles cost more in per-tile overhead and MMA latency than that saves: 11 % slower.)
   static constexpr int BN = 128;
+  static constexpr int P_COLS = BN * ELT / 4;            // TMEM columns of one tile's P (bf16 or e4m3, packed)
   // P overwrites S's first columns only when S, O and P of both tiles do not fit in 512 TMEM columns.
-  static constexpr bool ALIAS_P = (2 * BN + 2 * D + BN) > 512;
+  static constexpr bool ALIAS_P = (2 * BN + 2 * D + 2 * P_COLS) > 512;
   static constexpr int N_ISSUERS = ALIAS_P ? 1 : 2;
-  static constexpr int KCH = D / 64;                     // 128-byte column chunks per row
+  static constexpr int KCH = ROW_BYTES / 128;            // 128-byte column chunks per row
   static constexpr int Q_CHUNK = PF_BM * 128;            // 128 rows x 128 B
-  static constexpr int Q_TILE = KCH * Q_CHUNK;           // one 128 x D bf16 Q tile
+  static constexpr int Q_TILE = KCH * Q_CHUNK;           // one 128 x D Q tile
   static constexpr int KV_CHUNK = BN * 128;              // BN rows x 128 B
-  static constexpr int KV_TILE = KCH * KV_CHUNK;         // one BN x D bf16 K or V tile
+  static constexpr int KV_TILE = KCH * KV_CHUNK;         // one BN x D K or V tile
+  static constexpr int QK_STEPS = ROW_BYTES / 32;        // K-steps of Q K^T: 32 bytes (16 bf16 or 32 e4m3) each
+  static constexpr int PV_KEYS = 32 / ELT;               // keys per K-step of P V (8 TMEM columns of P)
   static constexpr int NST = (KV_TILE <= 16384) ? 8 : 4;  // K/V ring depth (each stage holds one tile)
   // Of every 8 exp2 pairs, how many use the FMA-pipe polynomial instead of the MUFU.  Off: measured inside
   // this kernel it costs more (issue slots, dependency chains) than the MUFU time it saves.
@@ -146,18 +153,18 @@ struct PfCfg {
   static constexpr int NBAR = 2 * NST + 2 + 4 + 2 * 6;
   static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + 2 * Q_TILE + NST * KV_TILE + NBAR * 8 +
                                     2 * (int)sizeof(PfItem) + PF_BM * 8 /*split merge*/ + 16;
-  // TMEM columns: S_t at BN*t, O_t at TM_O + D*t, P_t at TM_P + (BN/2)*t (or S_t's first columns if ALIAS_P)
+  // TMEM columns: S_t at BN*t, O_t at TM_O + D*t, P_t at TM_P + P_COLS*t (or S_t's first columns if ALIAS_P)
   static constexpr uint32_t TM_O = 2 * BN;
   static constexpr uint32_t TM_P = 2 * BN + 2 * D;
-  static_assert(TM_P + (ALIAS_P ? 0 : BN) <= 512, "TMEM columns");
+  static_assert(TM_P + (ALIAS_P ? 0 : 2 * P_COLS) <= 512, "TMEM columns");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 };
 
 // Shared-memory carve-up, common to every role.  Every member is the base address plus a compile-time
 // offset, computed where it is used (nothing but the base stays live in registers).
-template <int D>
+template <int D, bool F8 = false>
 struct PfSmem {
-  using C = PfCfg<D>;
+  using C = PfCfg<D, F8>;
   static constexpr int OFF_KV = 2 * C::Q_TILE;
   static constexpr int OFF_BAR = OFF_KV + C::NST * C::KV_TILE;
   static constexpr int B_FULL = 0, B_EMPTY = C::NST, B_QFULL = 2 * C::NST, B_QEMPTY = B_QFULL + 1,
@@ -248,13 +255,13 @@ __device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int idx) {
 }
 
 // Control warpgroup: warp 0 fetches items and streams Q, K, V with TMA; warps 1-2 issue MMAs; warp 3 idles.
-template <int D, int MODE>
+template <int D, int MODE, bool F8 = false>
 __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CUtensorMap &tmK,
                                                 const CUtensorMap &tmV, const PrefillParams &p, uint8_t *smem,
                                                 uint32_t tmem, int warp, int lane) {
-  using C = PfCfg<D>;
+  using C = PfCfg<D, F8>;
   constexpr bool PACKED = (MODE != MODE_DENSE);
-  PfSmem<D> sm(smem);
+  PfSmem<D, F8> sm(smem);
   if (warp == 0) {
     // ================================================================ work fetcher + TMA producer
     if (lane == 0) {
@@ -353,8 +360,8 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
   } else if (warp == 1 || (!C::ALIAS_P && warp == 2)) {
     // ================================================================ MMA issuer(s)
     if (lane == 0) {
-      constexpr uint32_t ID_QK = idesc_bf16_f32(PF_BM, C::BN, false);
-      constexpr uint32_t ID_PV = idesc_bf16_f32(PF_BM, D, true);
+      constexpr uint32_t ID_QK = F8 ? idesc_e4m3_f32(PF_BM, C::BN, false) : idesc_bf16_f32(PF_BM, C::BN, false);
+      constexpr uint32_t ID_PV = F8 ? idesc_e4m3_f32(PF_BM, D, true) : idesc_bf16_f32(PF_BM, D, true);
       const uint32_t sQa = smem_u32(sm.sQ()), sKVa = smem_u32(sm.sKV());
       // S_t = Q_t K^T : K-steps of 16 elements = 32 bytes inside a 128-byte swizzled row.
       const uint64_t dQ = sdesc_sw128(sQa, 16, 1024), dKV = sdesc_sw128(sKVa, 16, 1024);
@@ -363,23 +370,30 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
         const uint64_t da = dQ + (uint64_t)((t * C::Q_TILE) >> 4);
         const uint64_t db = dKV + (uint64_t)((st * C::KV_TILE) >> 4);
         const uint32_t dt = tmem + (uint32_t)(C::BN * t);
-        eta_static_for<D / 16>([&](auto kk_c) {
+        eta_static_for<C::QK_STEPS>([&](auto kk_c) {
           constexpr int kk = decltype(kk_c)::value;
           constexpr uint32_t a_off = ((uint32_t)(kk >> 2) * C::Q_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
           constexpr uint32_t b_off = ((uint32_t)(kk >> 2) * C::KV_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
-          mma_ss_off<a_off, b_off>(dt, da, db, ID_QK, kk > 0 ? 1u : 0u);
+          if constexpr (F8)
+            mma_ss_off_f8<a_off, b_off>(dt, da, db, ID_QK, kk > 0 ? 1u : 0u);
+          else
+            mma_ss_off<a_off, b_off>(dt, da, db, ID_QK, kk > 0 ? 1u : 0u);
         });
       };
       // O_t += P_t V : K-steps of 16 keys = 8 TMEM columns of packed bf16 P, 16 rows (2048 B) of V.
       auto issue_pv = [&](int t, int st, bool acc) {
-        const uint32_t tP = C::ALIAS_P ? tmem + (uint32_t)(C::BN * t) : tmem + C::TM_P + (uint32_t)(C::BN / 2 * t);
+        const uint32_t tP = C::ALIAS_P ? tmem + (uint32_t)(C::BN * t) : tmem + C::TM_P + (uint32_t)(C::P_COLS * t);
         const uint64_t db = dV + (uint64_t)((st * C::KV_TILE) >> 4);
         const uint32_t dt = tmem + C::TM_O + (uint32_t)(D * t);
         const uint32_t acc0 = acc ? 1u : 0u;
-        eta_static_for<C::BN / 16>([&](auto kk_c) {
+        // K-step kk: PV_KEYS keys = 8 TMEM columns of P, PV_KEYS rows (PV_KEYS * 128 B) of V
+        eta_static_for<C::BN / C::PV_KEYS>([&](auto kk_c) {
           constexpr int kk = decltype(kk_c)::value;
-          constexpr uint32_t ta_off = 8u * kk, b_off = (2048u * kk) / 16u;
-          mma_ts_off<ta_off, b_off>(dt, tP, db, ID_PV, kk > 0 ? 1u : acc0);
+          constexpr uint32_t ta_off = 8u * kk, b_off = (uint32_t)(C::PV_KEYS * 128 * kk) / 16u;
+          if constexpr (F8)
+            mma_ts_off_f8<ta_off, b_off>(dt, tP, db, ID_PV, kk > 0 ? 1u : acc0);
+          else
+            mma_ts_off<ta_off, b_off>(dt, tP, db, ID_PV, kk > 0 ? 1u : acc0);
         });
       };
       // Counts over all items; each gives the phase of the barrier it tracks.  With one issuer per tile
@@ -615,13 +629,13 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
 // (quarter, lane) owns query row 32 quarter + lane of its tile (= its TMEM lane): per key tile it loads the
 // S row from TMEM, applies the mask, updates the running max and exp-sum, writes P (bf16) to TMEM and
 // rescales its O row when the max moved; per item it finally normalises O and stores O and lse.
-template <int D, int MODE>
+template <int D, int MODE, bool F8 = false>
 __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t *smem, uint32_t tmem, int warp,
                                                 int lane) {
-  using C = PfCfg<D>;
+  using C = PfCfg<D, F8>;
   constexpr bool HSTU = (MODE == MODE_HSTU);
   constexpr bool PACKED = (MODE != MODE_DENSE);
-  PfSmem<D> sm(smem);
+  PfSmem<D, F8> sm(smem);
   const int t = (warp - 4) >> 2;
   const int quarter = warp & 3;
   const int row = quarter * 32 + lane;
@@ -629,7 +643,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
   constexpr int BN = C::BN;
   const uint32_t tS = tmem + lane_addr + (uint32_t)(BN * t);
   const uint32_t tO = tmem + lane_addr + C::TM_O + (uint32_t)(D * t);
-  const uint32_t tP = C::ALIAS_P ? tS : tmem + lane_addr + C::TM_P + (uint32_t)(BN / 2 * t);
+  const uint32_t tP = C::ALIAS_P ? tS : tmem + lane_addr + C::TM_P + (uint32_t)(C::P_COLS * t);
   const bool causal = HSTU ? true : (p.causal != 0);
   int gj = 0;  // key tiles of Q tile t processed, over all items (phases of s_full, p_full, pv_done)
   bool ok = true;
@@ -665,7 +679,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
       const int k0 = (kv_lo + j) * BN;
       const bool need_mask = (k0 + BN > L) || (causal && k0 + BN - 1 > q_start);
       const int kmax = causal ? min(L - 1, qpos) - k0 : L - 1 - k0;  // last visible key, tile-local
-      uint32_t pk[BN / 2];
+      uint32_t pk[C::P_COLS];
       bool resc = false;
       float f = 1.f, rowsum = 0.f, m_new = m_used;
       if constexpr (!HSTU) {
@@ -691,6 +705,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
         const float msub = (m_new == -INFINITY) ? 0.f : m_new;
         const uint64_t cs2 = f2pack(p.scale_log2, p.scale_log2), nm2 = f2pack(-msub, -msub);
         uint64_t rs_a = f2pack(0.f, 0.f), rs_b = f2pack(0.f, 0.f);
+        float q0 = 0.f, q1 = 0.f;  // (F8) the previous pair, packed with the next one
         // p = 2^(s * scale_log2 - m): pairs with (i % 8) < POLY_PAIRS go to the FMA-pipe polynomial on
         // unmasked tiles, the rest (and every element of a masked tile) to the MUFU.
         auto exp_row = [&](auto use_poly) {
@@ -708,7 +723,14 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
             }
             if (i & 1) rs_b = add_x2(rs_b, f2pack(p0, p1));
             else rs_a = add_x2(rs_a, f2pack(p0, p1));
-            pk[i] = pack_bf16x2(p0, p1);
+            if constexpr (F8) {
+              // four keys per TMEM column: pairs 2m and 2m+1 go to column m
+              if (i & 1) pk[i >> 1] = pack_e4m3x4(q0, q1, p0, p1);
+              q0 = p0;
+              q1 = p1;
+            } else {
+              pk[i] = pack_bf16x2(p0, p1);
+            }
           }
         };
         if (need_mask) exp_row(std::false_type{});
@@ -749,7 +771,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
         }
       }
 #pragma unroll
-      for (int cc = 0; cc < BN / 64; ++cc) ETA_TMEM_ST_X32(tP + 32u * cc, (pk + 32 * cc));
+      for (int cc = 0; cc < C::P_COLS / 32; ++cc) ETA_TMEM_ST_X32(tP + 32u * cc, (pk + 32 * cc));
       if constexpr (!HSTU) {
         if (__any_sync(0xffffffffu, resc && j > 0)) {
           const uint64_t f2 = f2pack(f, f);
@@ -807,7 +829,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
         merge = true;
       }
     }
-    const float inv_l = HSTU ? 1.f : ((l_fin > 0.f) ? 1.f / l_fin : 0.f);
+    const float inv_l = HSTU ? 1.f : ((l_fin > 0.f) ? p.o_scale / l_fin : 0.f);
     const float w0 = a0 * inv_l, w1 = a1 * inv_l;
     const bool valid = qpos < L;
     const uint32_t tO1 = tmem + lane_addr + C::TM_O + (uint32_t)D;  // O_1 (read here only when merging)
@@ -864,14 +886,14 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
   }
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool F8 = false>
 __global__ void __launch_bounds__(PF_THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
-  using C = PfCfg<D>;
+  using C = PfCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  PfSmem<D> sm(smem);
+  PfSmem<D, F8> sm(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ------------------------------------------------------------------ setup
@@ -909,7 +931,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   // both sides.
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(PF_CTRL_REGS));
-    prefill_control<D, MODE>(tmQ, tmK, tmV, p, smem, tmem, warp, lane);
+    prefill_control<D, MODE, F8>(tmQ, tmK, tmV, p, smem, tmem, warp, lane);
     tc_fence_before();
     asm volatile("bar.sync 1, %0;" ::"n"(PF_THREADS) : "memory");
     if (warp == 1) {
@@ -918,7 +940,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(PF_SM_REGS));
-    prefill_softmax<D, MODE>(p, smem, tmem, warp, lane);
+    prefill_softmax<D, MODE, F8>(p, smem, tmem, warp, lane);
     tc_fence_before();
     asm volatile("bar.sync 1, %0;" ::"n"(PF_THREADS) : "memory");
   }

@@ -14,8 +14,8 @@ from __future__ import annotations
 import torch
 
 # Config ids follow the workload list: 1 tiny check, 2 prefill d=64, 3 prefill d=128 (+ N sweep),
-# 4 HSTU jagged, 5 decode, 6 decode over a paged cache with grouped query heads.
-TINY, PREFILL_D64, PREFILL_D128, HSTU_JAGGED, DECODE, DECODE_PAGED = 1, 2, 3, 4, 5, 6
+# 4 HSTU jagged, 5 decode, 6 decode over a paged cache with grouped query heads, 7 prefill on e4m3 inputs.
+TINY, PREFILL_D64, PREFILL_D128, HSTU_JAGGED, DECODE, DECODE_PAGED, PREFILL_FP8 = 1, 2, 3, 4, 5, 6, 7
 
 
 def _gen(device, seed: int) -> torch.Generator:
@@ -110,3 +110,19 @@ def paged_decode_inputs(config: int, B: int, Hq: int, Hkv: int, d: int, page_siz
         kp[mask] = float("nan")
         vp[mask] = float("nan")
     return q, kp, vp, table, lens
+
+
+def fp8_dense_qkv(config: int, B: int, H: int, N: int, d: int, std: float = 1.0, device="cpu"):
+    """Q, K, V as e4m3 (torch.float8_e4m3fn) ``[B,H,N,d]`` with one descale factor per tensor: iid N(0, std^2)
+    values x are divided by amax(|x|) / 448 (the e4m3 maximum) and rounded to e4m3; the factor is returned so
+    that x ~ x8 * descale.  Returns (q8, k8, v8, (q_descale, k_descale, v_descale))."""
+    base = 1000 * config
+    out, scales = [], []
+    for i in range(3):
+        x = torch.randn(B, H, N, d, generator=_gen(device, base + i), device=device, dtype=torch.float32)
+        if std != 1.0:
+            x.mul_(std)
+        descale = float(x.abs().max()) / 448.0
+        out.append((x / descale).to(torch.float8_e4m3fn))
+        scales.append(descale)
+    return out[0], out[1], out[2], tuple(scales)

@@ -104,6 +104,21 @@ ETA_API int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o
                     void *stream);
 
 /*
+ * attn_fwd_fp8 -- attn_fwd with 8-bit inputs ("FlashAttention (TH)", section "FlashAttention-3": FP8 support).
+ * The pages give no scaling recipe; this one is per tensor: the caller passes q8, k8, v8 holding e4m3 values
+ * (torch.float8_e4m3fn, one byte each, [B, H, N, d]) and positive descale factors with Q = q8 * q_descale,
+ * K = k8 * k_descale, V = v8 * v_descale.  Then
+ *   s_ij = scale * q_descale * k_descale * (q8_i . k8_j)   (exact products, fp32 accumulation),
+ *   o_i  = v_descale * sum_j P8_ij v8_j / sum_j P_ij,  P_ij = e^(s_ij - m_i) as fp32, P8 its e4m3 rounding
+ *          (nearest; the P . V product runs on e4m3 operands), lse_i as in attn_fwd.
+ *   d must be 128 (a row is one 128-byte span); o bf16 or fp32 (o_dtype); lse fp32 or NULL.
+ * Errors as attn_fwd; ETA_ERR_HEAD_DIM for d != 128, ETA_ERR_ARG for a non-finite or non-positive descale.
+ */
+ETA_API int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N,
+                         int d, float scale, float q_descale, float k_descale, float v_descale, int causal,
+                         int o_dtype, void *stream);
+
+/*
  * hstu_fwd_jagged -- HSTU pointwise attention over S packed sequences:
  *   x_ij = alpha * q_i . k_j ;  p_ij = silu(x_ij) * inv_n  for j <= i (local indices), 0 otherwise ;
  *   o_i = sum_j p_ij v_j.

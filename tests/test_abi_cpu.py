@@ -108,3 +108,13 @@ def test_paged_decode_host_validation(L):
     assert call(wsz=ws - 1) == -5
     rc = call()
     assert rc in (-6, -8)
+
+
+def test_fp8_host_validation(L):
+    # (q, k, v, o, lse, B, H, N, d, scale, q_descale, k_descale, v_descale, causal, o_dtype, stream)
+    assert L.attn_fwd_fp8(NUL, A, A, A, NUL, 1, 1, 128, 128, 0.088, 1.0, 1.0, 1.0, 0, 0, S) == -1
+    assert L.attn_fwd_fp8(A, A, A, A, NUL, 1, 1, 128, 64, 0.088, 1.0, 1.0, 1.0, 0, 0, S) == -2
+    assert L.attn_fwd_fp8(A, A, A, A, NUL, 1, 1, 128, 128, 0.088, 0.0, 1.0, 1.0, 0, 0, S) == -7
+    assert L.attn_fwd_fp8(A, A, A, A, NUL, 1, 1, 128, 128, 0.088, 1.0, 1.0, float("inf"), 0, 0, S) == -7
+    assert L.attn_fwd_fp8(A, MIS, A, A, NUL, 1, 1, 128, 128, 0.088, 1.0, 1.0, 1.0, 0, 0, S) == -4
+    assert L.attn_fwd_fp8(A, A, A, A, NUL, 1, 1, 128, 128, 0.088, 1.0, 1.0, 1.0, 0, 0, S) in (-6, -8)
