@@ -497,6 +497,7 @@ CASES = {
     "prefill_d64_b4": ("dense", dict(B=4, H=32, N=4096, d=64)),
     "prefill_d128_b2": ("dense", dict(B=2, H=32, N=4096, d=128)),
     "prefill_d256_b2": ("dense", dict(B=2, H=16, N=4096, d=256)),
+    "prefill_fp8_b2": ("fp8", dict(B=2, H=32, N=4096, d=128)),
     "hstu_jagged": ("hstu", dict(S=16, H=4, d=64)),
     "decode_b2": ("decode", dict(B=2, H=32, d=128, Lmax=32768)),
     "decode_paged_b4": ("decode_paged", dict(B=4, Hq=32, Hkv=8, d=128, ps=64)),
@@ -516,6 +517,10 @@ def run_case(args):
         q, k, v = inputs.dense_qkv(inputs.PREFILL_D64 if s["d"] == 64 else inputs.PREFILL_D128, s["B"], s["H"],
                                    s["N"], s["d"], device=dev)
         fns = [lambda: eta.attn_fwd(q, k, v, causal=False), lambda: eta.attn_fwd(q, k, v, causal=True)]
+    elif kind == "fp8":
+        q8, k8, v8, (dq, dk, dv) = inputs.fp8_dense_qkv(inputs.PREFILL_FP8, s["B"], s["H"], s["N"], s["d"], device=dev)
+        fns = [lambda: eta.attn_fwd_fp8(q8, k8, v8, dq, dk, dv, causal=False),
+               lambda: eta.attn_fwd_fp8(q8, k8, v8, dq, dk, dv, causal=True)]
     elif kind == "hstu":
         lens = inputs.uniform_lengths(inputs.HSTU_JAGGED, s["S"], 256, 4096)
         cu = inputs.cu_seqlens(lens).to(dev)
