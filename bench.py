@@ -425,6 +425,17 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
                                                   "frac_of_peak": tf / pk}
         del q, k, v, o
 
+    # head dim 96 (rows of 192 B: one and a half swizzle chunks), the d=128 line's shape B8 H32 N4096 causal
+    B_, H_, N_ = 8, 32, 4096
+    q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, B_, H_, N_, 96, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B_, H_, N_), dtype=torch.float32, device=dev)
+    ms, _ = timed_steps(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse), K, W, flush, stream, ctx)
+    tf = 2.0 * B_ * H_ * N_ * N_ * 96 * K / (ctx.max(ms) * 1e-3) / 1e12
+    out["prefill_B8_H32_N4096_d96_causal"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+                                              "frac_of_peak": tf / pk}
+    del q, k, v, o, lse
+
     # head dim 256 (the FlashAttention-2 head size), B4 H16 N4096 causal: the same H*d as the d=128 line
     B_, H_, N_ = 4, 16, 4096
     q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, B_, H_, N_, 256, device=dev)
@@ -496,6 +507,7 @@ CASES = {
     "prefill_d64_headline": ("dense", dict(B=1, H=32, N=4096, d=64)),
     "prefill_d64_b4": ("dense", dict(B=4, H=32, N=4096, d=64)),
     "prefill_d128_b2": ("dense", dict(B=2, H=32, N=4096, d=128)),
+    "prefill_d96_b2": ("dense", dict(B=2, H=32, N=4096, d=96)),
     "prefill_d256_b2": ("dense", dict(B=2, H=16, N=4096, d=256)),
     "prefill_fp8_b2": ("fp8", dict(B=2, H=32, N=4096, d=128)),
     "hstu_jagged": ("hstu", dict(S=16, H=4, d=64)),

@@ -159,8 +159,8 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   if (mode != eta::MODE_DENSE && !cu_seqlens) return ETA_ERR_NULL;
   if (f8 && d != 128) return ETA_ERR_HEAD_DIM;  // e4m3: one 128-byte swizzle span per row
   if (f8 && (!finite_pos(qk_descale) || !finite_pos(v_descale))) return ETA_ERR_ARG;
-  // head dims 64 and 128 (two 128-row Q tiles per work item); 256 for softmax attention (one Q tile per item)
-  if (d != 64 && d != 128 && !(d == 256 && mode != eta::MODE_HSTU)) return ETA_ERR_HEAD_DIM;
+  // head dims 64, 96 and 128 (two 128-row Q tiles per work item); 256 for softmax attention (one Q tile per item)
+  if (d != 64 && d != 96 && d != 128 && !(d == 256 && mode != eta::MODE_HSTU)) return ETA_ERR_HEAD_DIM;
   const long long rows_per_item = (d == 256) ? eta::PF_BM : 2 * eta::PF_BM;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ETA_ERR_ALIGN;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ETA_ERR_ALIGN;
@@ -239,6 +239,11 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
     if (mode == eta::MODE_DENSE) return launch_prefill<64, eta::MODE_DENSE>(q, k, v, packed, n1, n2, grid, p, st);
     if (mode == eta::MODE_VARLEN) return launch_prefill<64, eta::MODE_VARLEN>(q, k, v, packed, n1, n2, grid, p, st);
     return launch_prefill<64, eta::MODE_HSTU>(q, k, v, packed, n1, n2, grid, p, st);
+  }
+  if (d == 96) {
+    if (mode == eta::MODE_DENSE) return launch_prefill<96, eta::MODE_DENSE>(q, k, v, packed, n1, n2, grid, p, st);
+    if (mode == eta::MODE_VARLEN) return launch_prefill<96, eta::MODE_VARLEN>(q, k, v, packed, n1, n2, grid, p, st);
+    return launch_prefill<96, eta::MODE_HSTU>(q, k, v, packed, n1, n2, grid, p, st);
   }
   if (mode == eta::MODE_DENSE) return launch_prefill<128, eta::MODE_DENSE>(q, k, v, packed, n1, n2, grid, p, st);
   if (mode == eta::MODE_VARLEN) return launch_prefill<128, eta::MODE_VARLEN>(q, k, v, packed, n1, n2, grid, p, st);

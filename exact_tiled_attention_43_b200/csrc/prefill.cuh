@@ -134,10 +134,15 @@ struct PfCfg {
   // halved tiles cost more in per-tile overhead and MMA latency than that saves: 11 % slower.)
   static constexpr int BN = 128;
   static constexpr int P_COLS = BN * ELT / 4;            // TMEM columns of one tile's P (bf16 or e4m3, packed)
+  // 128-byte column chunks per row.  A row that is not a whole number of chunks (d = 96: 192 bytes) has its
+  // last chunk half filled by the TMA's zero fill past the tensor's inner extent; the MMAs never read the
+  // zeros (Q K^T stops at ROW_BYTES, P V has N = D).
+  static constexpr int KCH = (ROW_BYTES + 127) / 128;
+  // TMEM columns reserved per O tile: the head dim rounded up to whole chunks (d = 96 keeps 128).
+  static constexpr int O_COLS = KCH * 128 / ELT;
   // P overwrites S's first columns only when S, O and P of both tiles do not fit in 512 TMEM columns.
-  static constexpr bool ALIAS_P = (2 * BN + 2 * D + 2 * P_COLS) > 512;
+  static constexpr bool ALIAS_P = (2 * BN + 2 * O_COLS + 2 * P_COLS) > 512;
   static constexpr int N_ISSUERS = ALIAS_P ? 1 : 2;
-  static constexpr int KCH = ROW_BYTES / 128;            // 128-byte column chunks per row
   static constexpr int Q_CHUNK = PF_BM * 128;            // 128 rows x 128 B
   static constexpr int Q_TILE = KCH * Q_CHUNK;           // one 128 x D Q tile
   static constexpr int KV_CHUNK = BN * 128;              // BN rows x 128 B
@@ -153,10 +158,11 @@ struct PfCfg {
   static constexpr int NBAR = 2 * NST + 2 + 4 + 2 * 6;
   static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + 2 * Q_TILE + NST * KV_TILE + NBAR * 8 +
                                     2 * (int)sizeof(PfItem) + PF_BM * 8 /*split merge*/ + 16;
-  // TMEM columns: S_t at BN*t, O_t at TM_O + D*t, P_t at TM_P + P_COLS*t (or S_t's first columns if ALIAS_P)
+  // TMEM columns: S_t at BN*t, O_t at TM_O + O_COLS*t, P_t at TM_P + P_COLS*t (or S_t's first columns if ALIAS_P)
   static constexpr uint32_t TM_O = 2 * BN;
-  static constexpr uint32_t TM_P = 2 * BN + 2 * D;
+  static constexpr uint32_t TM_P = 2 * BN + 2 * O_COLS;
   static_assert(TM_P + (ALIAS_P ? 0 : 2 * P_COLS) <= 512, "TMEM columns");
+  static_assert(ROW_BYTES % 32 == 0 && D % 32 == 0 && D <= O_COLS, "head dim: whole K-steps and TMEM loads");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -384,7 +390,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
       auto issue_pv = [&](int t, int st, bool acc) {
         const uint32_t tP = C::ALIAS_P ? tmem + (uint32_t)(C::BN * t) : tmem + C::TM_P + (uint32_t)(C::P_COLS * t);
         const uint64_t db = dV + (uint64_t)((st * C::KV_TILE) >> 4);
-        const uint32_t dt = tmem + C::TM_O + (uint32_t)(D * t);
+        const uint32_t dt = tmem + C::TM_O + (uint32_t)(C::O_COLS * t);
         const uint32_t acc0 = acc ? 1u : 0u;
         // K-step kk: PV_KEYS keys = 8 TMEM columns of P, PV_KEYS rows (PV_KEYS * 128 B) of V
         eta_static_for<C::BN / C::PV_KEYS>([&](auto kk_c) {
@@ -642,7 +648,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
   const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
   constexpr int BN = C::BN;
   const uint32_t tS = tmem + lane_addr + (uint32_t)(BN * t);
-  const uint32_t tO = tmem + lane_addr + C::TM_O + (uint32_t)(D * t);
+  const uint32_t tO = tmem + lane_addr + C::TM_O + (uint32_t)(C::O_COLS * t);
   const uint32_t tP = C::ALIAS_P ? tS : tmem + lane_addr + C::TM_P + (uint32_t)(C::P_COLS * t);
   const bool causal = HSTU ? true : (p.causal != 0);
   int gj = 0;  // key tiles of Q tile t processed, over all items (phases of s_full, p_full, pv_done)
@@ -832,7 +838,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
     const float inv_l = HSTU ? 1.f : ((l_fin > 0.f) ? p.o_scale / l_fin : 0.f);
     const float w0 = a0 * inv_l, w1 = a1 * inv_l;
     const bool valid = qpos < L;
-    const uint32_t tO1 = tmem + lane_addr + C::TM_O + (uint32_t)D;  // O_1 (read here only when merging)
+    const uint32_t tO1 = tmem + lane_addr + C::TM_O + (uint32_t)C::O_COLS;  // O_1 (read here only when merging)
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
       float ov[32];

@@ -32,8 +32,9 @@
  *    hold a sequence longer than max_len, a pipeline wait that ran out of time) never trap: the kernel
  *    keeps every access in bounds, records the first such condition in a device status word and carries
  *    on or returns.  Read it with eta_status().
- *  - Head dimension d must be 64 or 128.  The arithmetic is bf16 x bf16 products accumulated in fp32
- *    (tensor cores); softmax statistics and lse are fp32.
+ *  - Head dimension d: 64, 96 or 128 for every prefill call, 256 for softmax attention (attn_fwd,
+ *    attn_fwd_varlen), 128 for the e4m3 call, 64 or 128 for decode.  The arithmetic is bf16 x bf16
+ *    products accumulated in fp32 (tensor cores); softmax statistics and lse are fp32.
  */
 #ifndef ETA_H_
 #define ETA_H_
@@ -53,7 +54,7 @@ extern "C" {
 /* Host-side error codes (negative) returned by the entry points. */
 #define ETA_OK 0
 #define ETA_ERR_NULL (-1)      /* a required pointer is NULL */
-#define ETA_ERR_HEAD_DIM (-2)  /* d is not 64 or 128 (or 256, for attn_fwd / attn_fwd_varlen) */
+#define ETA_ERR_HEAD_DIM (-2)  /* d is not one the call supports (see "Head dimension" above) */
 #define ETA_ERR_SHAPE (-3)     /* a size is <= 0, too large for 32-bit indexing, or inconsistent */
 #define ETA_ERR_ALIGN (-4)     /* a tensor pointer is not 16-byte aligned */
 #define ETA_ERR_WORKSPACE (-5) /* workspace smaller than attn_decode_workspace_size() */
@@ -81,8 +82,9 @@ extern "C" {
  *             may be NULL (not written)
  *   scale   : multiplies Q K^T before the softmax (1/sqrt(d) in the formula); finite and > 0
  *   causal  : 0 = every key; 1 = query i sees keys j <= i (top-left aligned, diagonal included)
- *   d       : 64, 128 or 256 (256 is the FlashAttention-2 head size, "FlashAttention (TH)", section
- *             "FlashAttention-2"; it runs one 128-row Q tile per work item, see prefill_wide.cuh)
+ *   d       : 64, 96, 128 or 256 (96 and 256 are among the head sizes of "FlashAttention (TH)", section
+ *             "FlashAttention-2"; 256 runs one 128-row Q tile per work item, see prefill_wide.cuh; a
+ *             96-element row is 1.5 swizzle chunks, the TMA zero-fills the other half chunk in shared memory)
  * Errors: ETA_ERR_NULL, ETA_ERR_HEAD_DIM, ETA_ERR_SHAPE (B,H,N <= 0 or B*H*N*d >= 2^31), ETA_ERR_ALIGN,
  *         ETA_ERR_ARG, ETA_ERR_DEVICE, ETA_ERR_CUDA.
  */

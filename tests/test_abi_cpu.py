@@ -46,7 +46,8 @@ S = ctypes.c_void_p(0)
 
 def test_attn_fwd_host_validation(L):
     assert L.attn_fwd(NUL, A, A, A, NUL, 1, 1, 128, 64, 0.125, 0, 0, S) == -1
-    assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 96, 0.125, 0, 0, S) == -2
+    for bad_d in (32, 80, 112, 160, 192):
+        assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, bad_d, 0.125, 0, 0, S) == -2
     assert L.attn_fwd(A, A, A, A, NUL, 0, 1, 128, 64, 0.125, 0, 0, S) == -3
     assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 0, 64, 0.125, 0, 0, S) == -3
     assert L.attn_fwd(A, A, MIS, A, NUL, 1, 1, 128, 64, 0.125, 0, 0, S) == -4
@@ -57,6 +58,9 @@ def test_attn_fwd_host_validation(L):
     # valid arguments without a usable GPU: a clean negative code, no crash
     rc = L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 64, 0.125, 0, 0, S)
     assert rc in (-6, -8)
+    # head dim 96: accepted by every prefill mode (past the head-dim check: only the missing GPU stops it)
+    assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 96, 0.125, 1, 0, S) in (-6, -8)
+    assert L.hstu_fwd_jagged(A, A, A, A, A, 2, 128, 256, 1, 96, 0.125, 1.0, S) in (-6, -8)
     # head dim 256: accepted for softmax attention (dense and packed), not for HSTU
     assert L.attn_fwd(A, A, A, A, NUL, 1, 1, 128, 256, 0.0625, 1, 0, S) in (-6, -8)
     assert L.attn_fwd_varlen(A, A, A, A, NUL, A, 2, 128, 256, 1, 256, 0.0625, 1, 0, S) in (-6, -8)

@@ -25,7 +25,7 @@ def test_tiny_config(causal, out_dtype):
     check_lse(lse, lse_ref, "tiny lse")
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1, 2, 17, 127, 128, 129, 255, 256, 257, 700])
 def test_ragged_lengths(d, causal, N):
@@ -112,7 +112,7 @@ def test_prefill_d128_sweep_sampled(N):
         check_lse(sl(lse)[:, :, rows], lse_ref, "sweep lse")
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 @pytest.mark.parametrize("causal", [False, True])
 def test_more_items_than_sms(d, causal):
     """B*H*blocks well above the SM count: persistent CTAs take several items each (of unequal work when
@@ -151,7 +151,7 @@ def test_repeated_launches_on_two_streams():
         assert torch.equal(lse, ref_lse)
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 @pytest.mark.parametrize("shape", [(1, 20, 2000), (1, 160, 200), (2, 74, 1000)])
 def test_split_tail_items(d, shape):
     """Non-causal launches whose last wave is at most half full split those items: one Q tile each, keys

@@ -13,7 +13,7 @@ DEV = "cuda"
 EDGE_LENS = [1, 127, 128, 129, 0, 255, 256, 257, 300, 2]
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 @pytest.mark.parametrize("causal", [False, True])
 def test_varlen_edge_lengths(d, causal):
     cu = inputs.cu_seqlens(EDGE_LENS)
@@ -46,7 +46,7 @@ def test_varlen_bad_cu_seqlens_sets_status():
     assert eta.status() == eta.ETA_DEV_BAD_CUSEQ
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 96, 128])
 @pytest.mark.parametrize("inv_n", [1.0 / 4096, 1.0])
 def test_hstu_edge_lengths(d, inv_n):
     cu = inputs.cu_seqlens(EDGE_LENS)
