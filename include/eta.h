@@ -82,9 +82,9 @@ extern "C" {
  *             may be NULL (not written)
  *   scale   : multiplies Q K^T before the softmax (1/sqrt(d) in the formula); finite and > 0
  *   causal  : 0 = every key; 1 = query i sees keys j <= i (top-left aligned, diagonal included)
- *   d       : 64, 96, 128 or 256 (96 and 256 are among the head sizes of "FlashAttention (TH)", section
- *             "FlashAttention-2"; 256 runs one 128-row Q tile per work item, see prefill_wide.cuh; a
- *             96-element row is 1.5 swizzle chunks, the TMA zero-fills the other half chunk in shared memory)
+ *   d       : 64, 96, 128 or 256 ("FlashAttention (TH)", section "FlashAttention-2", extends head sizes
+ *             up to 256; 256 runs one 128-row Q tile per work item, see prefill_wide.cuh; a 96-element row
+ *             is 1.5 swizzle chunks, the TMA zero-fills the other half chunk in shared memory)
  * Errors: ETA_ERR_NULL, ETA_ERR_HEAD_DIM, ETA_ERR_SHAPE (B,H,N <= 0 or B*H*N*d >= 2^31), ETA_ERR_ALIGN,
  *         ETA_ERR_ARG, ETA_ERR_DEVICE, ETA_ERR_CUDA.
  */
