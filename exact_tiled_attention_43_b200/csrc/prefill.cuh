@@ -747,21 +747,23 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
         rowsum = (r0a + r1a) + (r2a + r3a);
         f = resc ? ex2_approx(m_used - msub) : 1.f;  // 0 on the first tile
       } else {
-        // HSTU: p = inv_n * silu(alpha s) = h + h * tanh(alpha s / 2),  h = (alpha * inv_n / 2) s
+        // HSTU: p = inv_n * silu(alpha s) = h + h * tanh(alpha s / 2),  h = (alpha * inv_n / 2) s.
+        // Masked keys get s = 0 first, which gives p = 0 exactly (h = 0), so the pointwise loop is the same
+        // straight-line code for every tile.
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c > kmax) sr[c] = 0u;
+        }
         const uint64_t ha2 = f2pack(p.hstu_half_alpha, p.hstu_half_alpha), ho2 = f2pack(p.hstu_out, p.hstu_out);
 #pragma unroll
         for (int i = 0; i < BN / 2; ++i) {
-          const int c0 = 2 * i;
-          const uint64_t s2 = f2pack(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1]));
+          const uint64_t s2 = f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
           float y0, y1;
           f2unpack(mul_x2(s2, ha2), y0, y1);
           const uint64_t h2 = mul_x2(s2, ho2);
           float p0, p1;
           f2unpack(fma_x2(h2, f2pack(tanh_approx(y0), tanh_approx(y1)), h2), p0, p1);
-          if (need_mask) {
-            p0 = (c0 > kmax) ? 0.f : p0;
-            p1 = (c0 + 1 > kmax) ? 0.f : p1;
-          }
           pk[i] = pack_bf16x2(p0, p1);
         }
       }
