@@ -110,7 +110,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.005)
+            time.sleep(0.002)
 
     def __enter__(self):
         if self._ok:
@@ -379,23 +379,44 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
     K, W = max(3, min(args.steps, 20)), max(3, args.warmup)
     pk = peaks["bf16_tflops"]
 
+    def timed(fn):
+        # An idle half second first, so that a case does not inherit the power-capped clocks of the
+        # previous (possibly seconds-long) one.  Short cases run more steps (about 25 ms of timed work,
+        # the same count on every rank) so that the clock sampler sees them, while the long ones stay in
+        # the burst regime that the measured peak describes; the clocks are reported with each case.
+        # Returns the device time scaled to K steps (the callers divide by K).
+        torch.cuda.synchronize()
+        time.sleep(0.5)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            fn()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        est = ctx.max(a.elapsed_time(b))
+        k = int(min(2000, max(K, math.ceil(25.0 / max(est, 1e-3)))))
+        with ClockSampler(ctx.local) as clk:
+            ms, _ = timed_steps(fn, k, W, flush, stream, ctx)
+        return ms / k * K, clk.summary()
+
     # prefill d=128, B=8, causal
     q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, 8, 32, 4096, 128, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
-    ms, _ = timed_steps(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse), K, W, flush, stream, ctx)
+    ms, ck = timed(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse))
     f = attn_flops(8, 32, 4096, 128, True)
     tf = f * K / (ctx.max(ms) * 1e-3) / 1e12
-    out["prefill_B8_H32_N4096_d128_causal"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+    out["prefill_B8_H32_N4096_d128_causal"] = {"clocks": ck, "value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
                                                "frac_of_peak": tf / pk}
     del q, k, v, o, lse
     for N in (1024, 8192, 32768):
         q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, 1, 32, N, 128, device=dev)
         o = torch.empty_like(q)
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
-        ms, _ = timed_steps(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse), K, W, flush, stream, ctx)
+        ms, ck = timed(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse))
         tf = attn_flops(1, 32, N, 128, True) * K / (ctx.max(ms) * 1e-3) / 1e12
-        out[f"prefill_B1_H32_N{N}_d128_causal"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+        out[f"prefill_B1_H32_N{N}_d128_causal"] = {"clocks": ck, "value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
                                                    "frac_of_peak": tf / pk}
         del q, k, v, o, lse
 
@@ -405,10 +426,9 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
     T = int(lens.sum())
     q, k, v = inputs.jagged_qkv(inputs.HSTU_JAGGED, T, 4, 64, std=0.5, device=dev)
     o = torch.empty_like(q)
-    ms, _ = timed_steps(lambda: eta.hstu_fwd_jagged(q, k, v, cu, 4096, 0.125, 1.0 / 4096, out=o), K, W, flush,
-                        stream, ctx)
+    ms, ck = timed(lambda: eta.hstu_fwd_jagged(q, k, v, cu, 4096, 0.125, 1.0 / 4096, out=o))
     tf = hstu_flops(lens.tolist(), 4, 64) * K / (ctx.max(ms) * 1e-3) / 1e12
-    out["hstu_jagged_S16_H4_d64"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K, "frac_of_peak": tf / pk,
+    out["hstu_jagged_S16_H4_d64"] = {"clocks": ck, "value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K, "frac_of_peak": tf / pk,
                                      "T": T}
     del q, k, v, o
 
@@ -418,10 +438,9 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
         cu = inputs.cu_seqlens(lens).to(dev)
         q, k, v = inputs.jagged_qkv(inputs.HSTU_JAGGED, S_ * N_, 4, 64, std=0.5, device=dev)
         o = torch.empty_like(q)
-        ms, _ = timed_steps(lambda: eta.hstu_fwd_jagged(q, k, v, cu, N_, 0.125, 1.0 / N_, out=o), K, W, flush,
-                            stream, ctx)
+        ms, ck = timed(lambda: eta.hstu_fwd_jagged(q, k, v, cu, N_, 0.125, 1.0 / N_, out=o))
         tf = hstu_flops(lens.tolist(), 4, 64) * K / (ctx.max(ms) * 1e-3) / 1e12
-        out[f"hstu_dense_S{S_}_H4_N{N_}_d64"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+        out[f"hstu_dense_S{S_}_H4_N{N_}_d64"] = {"clocks": ck, "value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
                                                   "frac_of_peak": tf / pk}
         del q, k, v, o
 
@@ -430,9 +449,9 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
     q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, B_, H_, N_, 96, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((B_, H_, N_), dtype=torch.float32, device=dev)
-    ms, _ = timed_steps(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse), K, W, flush, stream, ctx)
+    ms, ck = timed(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse))
     tf = 2.0 * B_ * H_ * N_ * N_ * 96 * K / (ctx.max(ms) * 1e-3) / 1e12
-    out["prefill_B8_H32_N4096_d96_causal"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+    out["prefill_B8_H32_N4096_d96_causal"] = {"clocks": ck, "value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
                                               "frac_of_peak": tf / pk}
     del q, k, v, o, lse
 
@@ -441,9 +460,9 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
     q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, B_, H_, N_, 256, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((B_, H_, N_), dtype=torch.float32, device=dev)
-    ms, _ = timed_steps(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse), K, W, flush, stream, ctx)
+    ms, ck = timed(lambda: eta.attn_fwd(q, k, v, causal=True, out=o, lse=lse))
     tf = 2.0 * B_ * H_ * N_ * N_ * 256 * K / (ctx.max(ms) * 1e-3) / 1e12
-    out["prefill_B4_H16_N4096_d256_causal"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+    out["prefill_B4_H16_N4096_d256_causal"] = {"clocks": ck, "value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
                                                "frac_of_peak": tf / pk}
     del q, k, v, o, lse
 
@@ -452,10 +471,9 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
     q8, k8, v8, (dq, dk, dv) = inputs.fp8_dense_qkv(inputs.PREFILL_FP8, 8, 32, 4096, 128, device=dev)
     o = torch.empty((8, 32, 4096, 128), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((8, 32, 4096), dtype=torch.float32, device=dev)
-    ms, _ = timed_steps(lambda: eta.attn_fwd_fp8(q8, k8, v8, dq, dk, dv, causal=True, out=o, lse=lse), K, W, flush,
-                        stream, ctx)
+    ms, ck = timed(lambda: eta.attn_fwd_fp8(q8, k8, v8, dq, dk, dv, causal=True, out=o, lse=lse))
     tf = 2.0 * 8 * 32 * 4096 * 4096 * 128 * K / (ctx.max(ms) * 1e-3) / 1e12
-    out["prefill_fp8_B8_H32_N4096_d128_causal"] = {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
+    out["prefill_fp8_B8_H32_N4096_d128_causal"] = {"clocks": ck, "value": tf, "unit": "TFLOP/s", "ms_per_step": ms / K,
                                                    "frac_of_peak": tf / (2.0 * pk),
                                                    "peak_note": "e4m3 peak = 2 x measured bf16"}
     del q8, k8, v8, o, lse
@@ -468,11 +486,10 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
     ws = torch.empty(eta.attn_decode_workspace_size(B, H, Lmax, d), dtype=torch.uint8, device=dev)
     od = torch.empty((B, H, d), dtype=torch.bfloat16, device=dev)
     ld = torch.empty((B, H), dtype=torch.float32, device=dev)
-    ms, _ = timed_steps(lambda: eta.attn_decode(q, kc, vc, kl, workspace=ws, out=od, lse=ld), K, W, flush, stream,
-                        ctx)
+    ms, ck = timed(lambda: eta.attn_decode(q, kc, vc, kl, workspace=ws, out=od, lse=ld))
     nbytes = 2.0 * H * d * 2 * float(lens.sum()) + q.numel() * 2 + od.numel() * 2 + ld.numel() * 4
     gbs = nbytes * K / (ctx.max(ms) * 1e-3) / 1e9
-    out["decode_B64_H32_d128_L8k-32k"] = {"value": gbs, "unit": "GB/s", "ms_per_step": ms / K,
+    out["decode_B64_H32_d128_L8k-32k"] = {"clocks": ck, "value": gbs, "unit": "GB/s", "ms_per_step": ms / K,
                                           "frac_of_peak": gbs / peaks["hbm_gbs"], "bytes_per_step": nbytes}
     del q, kc, vc, ws
     torch.cuda.empty_cache()
@@ -488,12 +505,11 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
                      device=dev)
     od = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
     ld = torch.empty((B, Hq), dtype=torch.float32, device=dev)
-    ms, _ = timed_steps(lambda: eta.attn_decode_paged(q, kp, vp, table, kl, workspace=ws, out=od, lse=ld), K, W,
-                        flush, stream, ctx)
+    ms, ck = timed(lambda: eta.attn_decode_paged(q, kp, vp, table, kl, workspace=ws, out=od, lse=ld))
     nbytes = (2.0 * Hkv * d * 2 * float(lens.sum()) + q.numel() * 2 + od.numel() * 2 + ld.numel() * 4 +
               table.numel() * 4)
     gbs = nbytes * K / (ctx.max(ms) * 1e-3) / 1e9
-    out["decode_paged_gqa_B64_Hq32_Hkv8_d128_page64_L8k-32k"] = {
+    out["decode_paged_gqa_B64_Hq32_Hkv8_d128_page64_L8k-32k"] = {"clocks": ck,
         "value": gbs, "unit": "GB/s", "ms_per_step": ms / K, "frac_of_peak": gbs / peaks["hbm_gbs"],
         "bytes_per_step": nbytes}
     del q, kp, vp, ws
