@@ -153,11 +153,15 @@ struct PfCfg {
   // Of every 8 exp2 pairs, how many use the FMA-pipe polynomial instead of the MUFU.  Off: measured inside
   // this kernel it costs more (issue slots, dependency chains) than the MUFU time it saves.
   static constexpr int POLY_PAIRS = 0;
-  // barriers: full/empty per stage; q_full, q_empty; item_full[2], item_empty[2];
+  // barriers: full/empty per stage; q_full[2], q_empty[2]; item_full[2], item_empty[2];
   // per tile {s_full, s_free, p_full, pv_done, o_free, mma_done}
-  static constexpr int NBAR = 2 * NST + 2 + 4 + 2 * 6;
-  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + 2 * Q_TILE + NST * KV_TILE + NBAR * 8 +
+  static constexpr int NBAR = 2 * NST + 4 + 4 + 2 * 6;
+  static constexpr int SMEM_FIXED = 1024 /*alignment slack*/ + NST * KV_TILE + NBAR * 8 +
                                     2 * (int)sizeof(PfItem) + PF_BM * 8 /*split merge*/ + 16;
+  // Slots for the two Q tiles of an item: two where they fit (d = 64, e4m3), so that the next item's Q is
+  // loaded while the current item still runs and its first QK^T is ready when the softmax gets to it.
+  static constexpr int QSLOTS = (SMEM_FIXED + 4 * Q_TILE <= 227 * 1024) ? 2 : 1;
+  static constexpr int SMEM_BYTES = SMEM_FIXED + QSLOTS * 2 * Q_TILE;
   // TMEM columns: S_t at BN*t, O_t at TM_O + O_COLS*t, P_t at TM_P + P_COLS*t (or S_t's first columns if ALIAS_P)
   static constexpr uint32_t TM_O = 2 * BN;
   static constexpr uint32_t TM_P = 2 * BN + 2 * O_COLS;
@@ -171,10 +175,10 @@ struct PfCfg {
 template <int D, bool F8 = false>
 struct PfSmem {
   using C = PfCfg<D, F8>;
-  static constexpr int OFF_KV = 2 * C::Q_TILE;
+  static constexpr int OFF_KV = C::QSLOTS * 2 * C::Q_TILE;
   static constexpr int OFF_BAR = OFF_KV + C::NST * C::KV_TILE;
-  static constexpr int B_FULL = 0, B_EMPTY = C::NST, B_QFULL = 2 * C::NST, B_QEMPTY = B_QFULL + 1,
-                       B_ITEM_FULL = B_QEMPTY + 1, B_ITEM_EMPTY = B_ITEM_FULL + 2, B_S_FULL = B_ITEM_EMPTY + 2,
+  static constexpr int B_FULL = 0, B_EMPTY = C::NST, B_QFULL = 2 * C::NST, B_QEMPTY = B_QFULL + 2,
+                       B_ITEM_FULL = B_QEMPTY + 2, B_ITEM_EMPTY = B_ITEM_FULL + 2, B_S_FULL = B_ITEM_EMPTY + 2,
                        B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 2,
                        B_O_FREE = B_PV_DONE + 2, B_MMA_DONE = B_O_FREE + 2, B_END = B_MMA_DONE + 2;
   static_assert(B_END == C::NBAR, "barrier count");
@@ -185,13 +189,13 @@ struct PfSmem {
   uint8_t *base;
   __device__ explicit PfSmem(uint8_t *smem) : base(smem) {}
   __device__ __forceinline__ uint64_t *bar(int i) const { return reinterpret_cast<uint64_t *>(base + OFF_BAR) + i; }
-  __device__ __forceinline__ uint8_t *sQ() const { return base; }
+  __device__ __forceinline__ uint8_t *sQ(int slot) const { return base + slot * 2 * C::Q_TILE; }
   __device__ __forceinline__ uint8_t *sKV() const { return base + OFF_KV; }
   __device__ __forceinline__ uint64_t *full(int i) const { return bar(B_FULL + i); }          // TMA -> MMA
   __device__ __forceinline__ uint64_t *empty(int i) const { return bar(B_EMPTY + i); }        // MMA -> TMA
-  // Q tiles of the current item landed / every QK^T of the item completed (Q may be overwritten)
-  __device__ __forceinline__ uint64_t *q_full() const { return bar(B_QFULL); }
-  __device__ __forceinline__ uint64_t *q_empty() const { return bar(B_QEMPTY); }
+  // Q slot: the item's Q tiles landed / every QK^T of the item completed (the slot may be overwritten)
+  __device__ __forceinline__ uint64_t *q_full(int slot) const { return bar(B_QFULL + slot); }
+  __device__ __forceinline__ uint64_t *q_empty(int slot) const { return bar(B_QEMPTY + slot); }
   // item ring: published by the producer / read by every consumer warp
   __device__ __forceinline__ uint64_t *item_full(int i) const { return bar(B_ITEM_FULL + i); }
   __device__ __forceinline__ uint64_t *item_empty(int i) const { return bar(B_ITEM_EMPTY + i); }
@@ -308,23 +312,24 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
         sm.items()[k & 1] = it;
         mbar_arrive(sm.item_full(k & 1));  // release semantics: the item is visible to its readers
         if (it.stop) break;
-        // Q tiles: every QK^T of the previous item must have finished reading them.
-        if (k > 0) {
-          ok = mbar_wait(sm.q_empty(), (k - 1) & 1, sm.abort_flag(), p.wait_ns);
+        // Q tiles into slot k % QSLOTS: every QK^T of the item that used the slot before must have finished.
+        const int qs = k % C::QSLOTS;
+        if (k >= C::QSLOTS) {
+          ok = mbar_wait(sm.q_empty(qs), (k / C::QSLOTS - 1) & 1, sm.abort_flag(), p.wait_ns);
           if (!ok) break;
         }
-        mbar_arrive_expect_tx(sm.q_full(), 2 * C::Q_TILE);
+        mbar_arrive_expect_tx(sm.q_full(qs), 2 * C::Q_TILE);
         // Q tile t: rows r0 + 128 t (whole item), or the item's one Q tile in both slots (split item).
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           const int qrow = it.r0 + (it.split ? 0 : t * PF_BM);
 #pragma unroll
           for (int c = 0; c < C::KCH; ++c) {
-            uint8_t *dst = sm.sQ() + t * C::Q_TILE + c * C::Q_CHUNK;
+            uint8_t *dst = sm.sQ(qs) + t * C::Q_TILE + c * C::Q_CHUNK;
             if constexpr (PACKED)
-              tma_load_3d(dst, &tmQ, sm.q_full(), 64 * c, it.h, it.seq_start + qrow);
+              tma_load_3d(dst, &tmQ, sm.q_full(qs), 64 * c, it.h, it.seq_start + qrow);
             else
-              tma_load_3d(dst, &tmQ, sm.q_full(), 64 * c, qrow, it.bh);
+              tma_load_3d(dst, &tmQ, sm.q_full(qs), 64 * c, qrow, it.bh);
           }
         }
         ++q_issued;
@@ -358,7 +363,8 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
       if (!retired) retire();  // abandoned before the work ran out
       if (!ok) {
         // Abandoned pipeline: let copies already in flight land before shared memory is released.
-        if (q_issued > 0) mbar_wait(sm.q_full(), (q_issued - 1) & 1, nullptr, p.wait_ns);
+        for (int i = max(0, q_issued - C::QSLOTS); i < q_issued; ++i)
+          mbar_wait(sm.q_full(i % C::QSLOTS), (i / C::QSLOTS) & 1, nullptr, p.wait_ns);
         for (int i = max(0, kv_issued - C::NST); i < kv_issued; ++i)
           mbar_wait(sm.full(i % C::NST), (i / C::NST) & 1, nullptr, p.wait_ns);
       }
@@ -368,12 +374,13 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
     if (lane == 0) {
       constexpr uint32_t ID_QK = F8 ? idesc_e4m3_f32(PF_BM, C::BN, false) : idesc_bf16_f32(PF_BM, C::BN, false);
       constexpr uint32_t ID_PV = F8 ? idesc_e4m3_f32(PF_BM, D, true) : idesc_bf16_f32(PF_BM, D, true);
-      const uint32_t sQa = smem_u32(sm.sQ()), sKVa = smem_u32(sm.sKV());
+      const uint32_t sQa = smem_u32(sm.sQ(0)), sKVa = smem_u32(sm.sKV());
+      uint32_t q_off = 0;  // byte offset of the current item's Q slot
       // S_t = Q_t K^T : K-steps of 16 elements = 32 bytes inside a 128-byte swizzled row.
       const uint64_t dQ = sdesc_sw128(sQa, 16, 1024), dKV = sdesc_sw128(sKVa, 16, 1024);
       const uint64_t dV = sdesc_sw128(sKVa, C::KV_CHUNK, 1024);
       auto issue_s = [&](int t, int st) {
-        const uint64_t da = dQ + (uint64_t)((t * C::Q_TILE) >> 4);
+        const uint64_t da = dQ + (uint64_t)((q_off + (uint32_t)(t * C::Q_TILE)) >> 4);
         const uint64_t db = dKV + (uint64_t)((st * C::KV_TILE) >> 4);
         const uint32_t dt = tmem + (uint32_t)(C::BN * t);
         eta_static_for<C::QK_STEPS>([&](auto kk_c) {
@@ -416,7 +423,9 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
         mbar_arrive(sm.item_empty(k & 1));
         if (it.stop) break;
         const int n_t[2] = {it.n0, it.n1};
-        ok = mbar_wait(sm.q_full(), k & 1, sm.abort_flag(), p.wait_ns);
+        const int qs = k % C::QSLOTS;
+        q_off = (uint32_t)(qs * 2 * C::Q_TILE);
+        ok = mbar_wait(sm.q_full(qs), (k / C::QSLOTS) & 1, sm.abort_flag(), p.wait_ns);
         if (!ok) break;
         auto kv_wait = [&](int i) {  // item-local ring position i (numbered by kv_pos)
           const int g = kv_base + i;
@@ -443,7 +452,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
               mma_commit(sm.empty(kv_stage(0)));
               ++gs[0];
             }
-            if (nt <= 1) mma_commit(sm.q_empty());  // every QK^T of this item is issued
+            if (nt <= 1) mma_commit(sm.q_empty(qs));  // every QK^T of this item is issued
             for (int j = 0; ok && j < nt; ++j) {
               if (j + 1 < nt) {
                 ok = kv_wait(2 * j + 2) && mbar_wait(sm.s_free(t), (gs[0] - 1) & 1, sm.abort_flag(), p.wait_ns);
@@ -453,7 +462,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
                 mma_commit(sm.s_full(t));
                 mma_commit(sm.empty(kv_stage(2 * j + 2)));
                 ++gs[0];
-                if (j + 2 == nt) mma_commit(sm.q_empty());
+                if (j + 2 == nt) mma_commit(sm.q_empty(qs));
               }
               ok = kv_wait(2 * j + 1) && mbar_wait(sm.p_full(t), gp[0] & 1, sm.abort_flag(), p.wait_ns) &&
                    (j > 0 || o_wait(t, 0));
@@ -494,7 +503,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
               mma_commit(sm.empty(kv_stage(pk)));
               ++gs[0];
             }
-            if (nt <= 1) mma_commit(sm.q_empty());  // every QK^T of this item is issued
+            if (nt <= 1) mma_commit(sm.q_empty(qs));  // every QK^T of this item is issued
             for (int j = 0; ok && j < nt; ++j) {
               if (j + 1 < nt) {
                 const int pk = kv_pos(it, t, j + 1, 0);
@@ -508,7 +517,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
                 mma_commit(sm.s_full(t));
                 mma_commit(sm.empty(kv_stage(pk)));
                 ++gs[0];
-                if (j + 2 == nt) mma_commit(sm.q_empty());
+                if (j + 2 == nt) mma_commit(sm.q_empty(qs));
               }
               const int pv = kv_pos(it, t, j, 1);
               ok = kv_wait(pv);
@@ -545,7 +554,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
                 ++gs[t];
               }
             mma_commit(sm.empty(kv_stage(0)));
-            if (n_kv == 1) mma_commit(sm.q_empty());
+            if (n_kv == 1) mma_commit(sm.q_empty(qs));
             for (int j = 0; ok && j < n_kv; ++j) {
               ok = kv_wait(2 * j + 1);
               if (!ok) break;
@@ -573,7 +582,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
               if (!ok) break;
               mma_commit(sm.empty(kv_stage(2 * j + 1)));
               if (k_ready) mma_commit(sm.empty(kv_stage(2 * j + 2)));
-              if (j + 2 == n_kv) mma_commit(sm.q_empty());
+              if (j + 2 == n_kv) mma_commit(sm.q_empty(qs));
             }
           } else {
             // Split item: every ring position serves one tile (both tiles have key tiles).
@@ -589,7 +598,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
               ++gs[t];
             }
             if (!ok) break;
-            if (n_kv == 1) mma_commit(sm.q_empty());
+            if (n_kv == 1) mma_commit(sm.q_empty(qs));
             for (int j = 0; ok && j < n_kv; ++j) {
 #pragma unroll
               for (int t = 0; t < 2; ++t) {
@@ -614,7 +623,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
                 }
               }
               if (!ok) break;
-              if (j + 2 == n_kv) mma_commit(sm.q_empty());
+              if (j + 2 == n_kv) mma_commit(sm.q_empty(qs));
             }
           }
 #pragma unroll
@@ -910,8 +919,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       mbar_init(sm.full(i), 1);
       mbar_init(sm.empty(i), C::N_ISSUERS);  // released by each MMA issuer
     }
-    mbar_init(sm.q_full(), 1);
-    mbar_init(sm.q_empty(), C::N_ISSUERS);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(sm.q_full(i), 1);
+      mbar_init(sm.q_empty(i), C::N_ISSUERS);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(sm.item_full(i), 1);
       mbar_init(sm.item_empty(i), C::N_ISSUERS + PF_SM_WARPS);  // every consumer warp reads the item
