@@ -30,10 +30,13 @@
 //   warp 3      no role.
 //   warps 4-11  two softmax warpgroups, one per Q tile; thread r owns query row r = TMEM lane r.
 //
-// TMEM (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D).
+// TMEM (512 columns x 128 lanes): S_0 [0,128), S_1 [128,256), O_t at 256 + t * O_COLS (O_COLS = D rounded up
+// to whole 64-column chunks: 64 for D = 64, 128 for D = 96 and 128).
 //   D = 64: P_t has its own columns [384+64t, 448+64t); issuer 1+t serves Q tile t and issues the next
-//           S_t as soon as the softmax has copied S_t to registers.
-//   D = 128: TMEM is full; P_t overwrites the first 64 columns of S_t and one issuer (warp 1) runs
+//           S_t as soon as the softmax has copied S_t to registers.  Two Q slots in shared memory: the
+//           next item's Q tiles load while the current item runs.
+//   D = 96, 128 (and e4m3 at 128): TMEM is full; P_t overwrites the first columns of S_t and one issuer
+//           (warp 1) runs
 //           PV_0(j), S_0(j+1), PV_1(j), S_1(j+1) with no wait between a PV and the next QK^T: tcgen05.mma
 //           operations issued by one thread execute in issue order, so the QK^T's writes follow the PV's
 //           reads of P, and the QK^T's commit also covers the PV (a softmax that has seen the new S may
