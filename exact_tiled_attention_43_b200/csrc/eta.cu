@@ -204,18 +204,29 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   if (rc != ETA_OK) return rc;
   int sms = 0;
   if ((rc = sm_count(&sms)) != ETA_OK) return rc;
-  const long long G = std::min<long long>(n_items, sms);
-  const dim3 grid((unsigned)G, 1, 1);  // persistent: at most one CTA per SM
-  // Dense non-causal items all cost the same.  When their count leaves a last wave at most half full, those
-  // last items are split in two (one Q tile each, keys halved between the CTA's two softmax warpgroups), so
-  // the last wave takes about half an item's time.  Needs at least two key tiles (N > 128).
+  const long long G = std::min<long long>(n_items, sms);  // CTAs the unsplit items would occupy
+  // Split items (softmax modes): one Q tile each, its key tiles halved between the CTA's two softmax
+  // warpgroups and merged in the CTA (needs at least two key tiles: more than 128 rows).  Non-causal dense
+  // items all cost the same: when their count leaves a last wave at most half full, those last items are
+  // split, so the last wave takes about half an item's time.  At d = 64, launches too small to fill the
+  // GPU split every item: non-causal ones with at most half as many items as SMs, causal ones (whose
+  // heaviest item sets the time of a single partial wave) with no more items than SMs.  (At d = 128 a split
+  // item streams twice the K/V bytes per key step -- its tiles serve one warpgroup each -- and measured
+  // no faster there.)  Packed (varlen) launches follow the same rules on their item count.
   long long n_whole = n_items;
-  if (mode == eta::MODE_DENSE && causal == 0 && d <= 128 && N > 128 && n_items > G) {
-    const long long R = n_items % G;
-    if (R > 0 && 2 * R <= G) n_whole = n_items - R;
+  const int rows = (mode == eta::MODE_DENSE) ? N : max_len;
+  if (mode != eta::MODE_HSTU && d <= 128 && rows > 128) {
+    if (causal == 0 && n_items > G) {
+      const long long R = n_items % G;
+      if (R > 0 && 2 * R <= G) n_whole = n_items - R;
+    } else if (d == 64 && ((causal == 0 && 2 * n_items <= sms) || (causal != 0 && n_items <= sms))) {
+      n_whole = 0;
+    }
   }
   p.n_whole = (int)n_whole;
   p.n_items = (int)(n_whole + 2 * (n_items - n_whole));
+  // persistent: at most one CTA per SM, and no more CTAs than (split) items
+  const dim3 grid((unsigned)std::min<long long>(p.n_items, sms), 1, 1);
   p.sched_slot = next_sched_slot();
   p.o = o;
   p.lse = (mode == eta::MODE_HSTU) ? nullptr : lse;

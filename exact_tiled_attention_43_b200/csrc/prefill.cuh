@@ -226,7 +226,7 @@ __device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int idx) {
   constexpr int BN = PfCfg<D>::BN;
   PfItem it{};
   int half = -1;
-  if (idx >= p.n_whole) {  // split halves (only dense non-causal launches with N > 128 have any)
+  if (idx >= p.n_whole) {  // split halves (only softmax launches with rows > 128 have any)
     half = (idx - p.n_whole) & 1;
     idx = p.n_whole + ((idx - p.n_whole) >> 1);
   }
@@ -258,10 +258,12 @@ __device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int idx) {
   it.split = 0;
   it.stop = 0;
   if (half >= 0) {
-    const int n = (it.L + BN - 1) / BN;  // >= 2
-    it.split = 1;
+    // One Q tile (rows r0 + 128 half) whose key tiles are halved between the warpgroups.  Causal: the keys up
+    // to the tile's diagonal; a tile that sees a single key tile stays whole (its second tile empty).
     it.r0 += half * PF_BM;
-    it.n0 = (n + 1) / 2;
+    const int n = ((causal ? min(it.L, it.r0 + PF_BM) : it.L) + BN - 1) / BN;
+    it.split = (n >= 2) ? 1 : 0;
+    it.n0 = (n + it.split) >> it.split;  // (n + 1) / 2 when split, else n
     it.n1 = n - it.n0;
   }
   return it;
@@ -444,7 +446,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
           // ---------------- issuer 1+t serves Q tile t; the next S_t as soon as S_t is free
           const int t = warp - 1;
           const int nt = (t == 0) ? it.n0 : it.n1;
-          if (MODE != MODE_DENSE || !it.split) {
+          if (MODE == MODE_HSTU || !it.split) {
             const int n_kv = max(it.n0, it.n1);
             if (nt > 0) {
               ok = kv_wait(0) && (gs[0] == 0 || mbar_wait(sm.s_free(t), (gs[0] - 1) & 1, sm.abort_flag(), p.wait_ns));
@@ -545,7 +547,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
           // ---------------- one issuer for both tiles; P aliased into S; issue order PV_t(j), S_t(j+1).
           // A whole item's K_j / V_j serve both tiles (released after both); a split item's each serve one.
           const int n_kv = max(it.n0, it.n1);  // >= 1: an item has at least one row
-          if (MODE != MODE_DENSE || !it.split) {
+          if (MODE == MODE_HSTU || !it.split) {
             ok = kv_wait(0);
             if (!ok) break;
             tc_fence_after();
@@ -829,7 +831,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
     //   m = max(m0, m1),  l = l0 2^(m0-m) + l1 2^(m1-m),  O = (O_0 2^(m0-m) + O_1 2^(m1-m)) / l.
     float m_fin = m_used, l_fin = l, a0 = 1.f, a1 = 0.f;
     bool merge = false;
-    if constexpr (MODE == MODE_DENSE) {
+    if constexpr (MODE != MODE_HSTU) {
       if (it.split) {
         if (t == 1) {
           // Hand this row's (m, l) to the first warpgroup, which reads O_1 from TMEM and stores the row.

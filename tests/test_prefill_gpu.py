@@ -127,6 +127,25 @@ def test_more_items_than_sms(d, causal):
     check_lse(lse, lse_ref, "items>SMs lse")
 
 
+@pytest.mark.parametrize("d", [64, 96, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", [(1, 32, 1024), (1, 16, 1500), (1, 8, 2048), (3, 1, 700)])
+def test_split_all_items(d, causal, shape):
+    """Launches too small to fill the GPU: at d = 64 causal ones with no more items than SMs split every item
+    (one Q tile, its keys up to the diagonal halved between the warpgroups; a Q tile that sees one key tile
+    stays whole), non-causal ones with at most half as many items as SMs too; d = 96 and 128 run the same
+    shapes unsplit.  (1,32,1024): 128 items; (1,16,1500): 96, ragged; (1,8,2048): 64; (3,1,700): 9, ragged.
+    Every row compared, fp32 output."""
+    B, H, N = shape
+    q, k, v = (t.to(DEV) for t in inputs.dense_qkv(14, B, H, N, d))
+    scale = eta.default_scale(d)
+    o, lse = eta.attn_fwd(q, k, v, causal=causal, scale=scale, out_dtype=torch.float32)
+    assert eta.status() == 0
+    o_ref, lse_ref = oracle.attn(q, k, v, scale, causal)
+    check_o(o, o_ref, f"split all {shape} d={d} causal={causal}")
+    check_lse(lse, lse_ref, "split all lse")
+
+
 def test_repeated_launches_on_two_streams():
     """Hundreds of launches in a row, alternating between two streams, reuse every work-counter slot more
     than once: each result must be bit-identical to the first (an item's arithmetic does not depend on
