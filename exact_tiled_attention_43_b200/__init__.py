@@ -41,6 +41,8 @@ SIGNATURES = {
     "eta_strerror": (ctypes.c_char_p, [_I]),
     "eta_set_wait_timeout_ns": (None, [_LL]),
     "eta_selftest_wait_timeout": (_I, [_VP]),
+    "eta_prefill_plan": (_I, [_I, _LL, _LL, _I, _I, _I, ctypes.POINTER(ctypes.c_longlong),
+                              ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_int)]),
 }
 
 
@@ -62,6 +64,20 @@ def lib():
             fn.argtypes = args
         _lib = L
     return _lib
+
+
+PLAN_KINDS = {"dense": 0, "varlen": 1, "hstu": 2}
+
+
+def prefill_plan(kind: str, units: int, rows: int, d: int, causal: bool, sms: int):
+    """The work decomposition a prefill call would launch on a GPU with `sms` SMs (host logic, no GPU):
+    (work items, items run whole, CTAs of the persistent grid).  kind: "dense", "varlen" or "hstu";
+    units = B*H or S*H; rows = N or max_len."""
+    items, whole, ctas = ctypes.c_longlong(), ctypes.c_longlong(), ctypes.c_int()
+    rc = lib().eta_prefill_plan(PLAN_KINDS[kind], int(units), int(rows), int(d), int(bool(causal)), int(sms),
+                                ctypes.byref(items), ctypes.byref(whole), ctypes.byref(ctas))
+    _check(rc, "eta_prefill_plan")
+    return items.value, whole.value, ctas.value
 
 
 def strerror(code: int) -> str:

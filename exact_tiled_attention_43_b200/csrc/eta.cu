@@ -151,6 +151,46 @@ int launch_prefill(const void *q, const void *k, const void *v, bool packed, lon
 
 bool finite_pos(float x) { return std::isfinite(x) && x > 0.f; }
 
+// Work decomposition of a prefill launch: `units` (batch, head) or (sequence, head) pairs of `rows` query
+// rows (N, or max_len for packed launches) -> work items, how many stay whole, and the persistent grid.
+struct PrefillPlan {
+  long long nblk = 0, items = 0, whole = 0, split_items = 0;
+  int ctas = 0;
+};
+int plan_prefill(int mode, long long units, long long rows, int d, int causal, int sms, PrefillPlan *pl) {
+  if (d != 64 && d != 96 && d != 128 && !(d == 256 && mode != eta::MODE_HSTU)) return ETA_ERR_HEAD_DIM;
+  if (units <= 0 || rows <= 0 || sms <= 0) return ETA_ERR_SHAPE;
+  if (causal != 0 && causal != 1) return ETA_ERR_ARG;
+  const long long rows_per_item = (d == 256) ? eta::PF_BM : 2 * eta::PF_BM;  // one or two 128-row Q tiles
+  pl->nblk = (rows + rows_per_item - 1) / rows_per_item;
+  if (pl->nblk > 65535) return ETA_ERR_SHAPE;
+  pl->items = units * pl->nblk;
+  // The work counter may run past the work count by one per CTA: keep it far from 2^32.
+  if (pl->items > (long long)INT_MAX / 4) return ETA_ERR_SHAPE;
+  const long long G = std::min<long long>(pl->items, sms);  // CTAs the unsplit items would occupy
+  // Split items (softmax modes): one Q tile each, its key tiles halved between the CTA's two softmax
+  // warpgroups and merged in the CTA (needs at least two key tiles: more than 128 rows).  Non-causal dense
+  // items all cost the same: when their count leaves a last wave at most half full, those last items are
+  // split, so the last wave takes about half an item's time.  At d = 64, launches too small to fill the
+  // GPU split every item: non-causal ones with at most half as many items as SMs, causal ones (whose
+  // heaviest item sets the time of a single partial wave) with no more items than SMs.  (At d = 128 a split
+  // item streams twice the K/V bytes per key step -- its tiles serve one warpgroup each -- and measured
+  // no faster there.)  Packed (varlen) launches follow the same rules on their item count.
+  pl->whole = pl->items;
+  if (mode != eta::MODE_HSTU && d <= 128 && rows > 128) {
+    if (causal == 0 && pl->items > G) {
+      const long long R = pl->items % G;
+      if (R > 0 && 2 * R <= G) pl->whole = pl->items - R;
+    } else if (d == 64 && ((causal == 0 && 2 * pl->items <= sms) || (causal != 0 && pl->items <= sms))) {
+      pl->whole = 0;
+    }
+  }
+  pl->split_items = pl->whole + 2 * (pl->items - pl->whole);
+  // persistent: at most one CTA per SM, and no more CTAs than (split) items
+  pl->ctas = (int)std::min<long long>(pl->split_items, sms);
+  return ETA_OK;
+}
+
 int prefill_common(int mode, const void *q, const void *k, const void *v, void *o, float *lse,
                    const int *cu_seqlens, int B, int S, int N, int max_len, int T_total, int H, int d,
                    float scale, int causal, int o_dtype, float alpha, float inv_n, void *stream, bool f8 = false,
@@ -161,72 +201,49 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   if (f8 && (!finite_pos(qk_descale) || !finite_pos(v_descale))) return ETA_ERR_ARG;
   // head dims 64, 96 and 128 (two 128-row Q tiles per work item); 256 for softmax attention (one Q tile per item)
   if (d != 64 && d != 96 && d != 128 && !(d == 256 && mode != eta::MODE_HSTU)) return ETA_ERR_HEAD_DIM;
-  const long long rows_per_item = (d == 256) ? eta::PF_BM : 2 * eta::PF_BM;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ETA_ERR_ALIGN;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ETA_ERR_ALIGN;
   if (o_dtype != ETA_OUT_BF16 && o_dtype != ETA_OUT_F32) return ETA_ERR_ARG;
   if (causal != 0 && causal != 1) return ETA_ERR_ARG;
   if (H <= 0 || H > 65535) return ETA_ERR_SHAPE;
   eta::PrefillParams p{};
-  long long n1, n2, n_items;
+  long long n1, n2, units, rows;
   if (mode == eta::MODE_DENSE) {
     if (B <= 0 || N <= 0) return ETA_ERR_SHAPE;
-    const long long bh = (long long)B * H;
-    const long long nblk = ((long long)N + rows_per_item - 1) / rows_per_item;
-    if (bh > INT_MAX || nblk > 65535) return ETA_ERR_SHAPE;
-    n_items = bh * nblk;
+    units = (long long)B * H;
+    if (units > INT_MAX) return ETA_ERR_SHAPE;
+    rows = N;
     n1 = N;
-    n2 = bh;
+    n2 = units;
     p.N = N;
-    p.BH = (int)bh;
-    p.nblk = (int)nblk;
+    p.BH = (int)units;
   } else {
     if (S <= 0 || max_len <= 0 || T_total < 0 || S > 65535) return ETA_ERR_SHAPE;
     if (T_total == 0) return ETA_OK;  // nothing to compute
-    const long long nblk = ((long long)max_len + rows_per_item - 1) / rows_per_item;
-    if (nblk > 65535) return ETA_ERR_SHAPE;
-    n_items = (long long)S * H * nblk;
+    units = (long long)S * H;
+    rows = max_len;
     n1 = H;
     n2 = T_total;
     p.max_len = max_len;
     p.S = S;
-    p.nblk = (int)nblk;
   }
-  // The work counter may run past the work count by one per CTA: keep it far from 2^32.
-  if (n_items > (long long)INT_MAX / 2) return ETA_ERR_SHAPE;
   if (mode == eta::MODE_HSTU) {
     if (!std::isfinite(alpha) || !finite_pos(inv_n)) return ETA_ERR_ARG;
     if (o_dtype != ETA_OUT_BF16) return ETA_ERR_ARG;
   } else if (!finite_pos(scale)) {
     return ETA_ERR_ARG;
   }
-  int rc = check_device();
+  PrefillPlan pl;
+  int rc = plan_prefill(mode, units, rows, d, causal, 1, &pl);  // shape checks before any device query
   if (rc != ETA_OK) return rc;
+  if ((rc = check_device()) != ETA_OK) return rc;
   int sms = 0;
   if ((rc = sm_count(&sms)) != ETA_OK) return rc;
-  const long long G = std::min<long long>(n_items, sms);  // CTAs the unsplit items would occupy
-  // Split items (softmax modes): one Q tile each, its key tiles halved between the CTA's two softmax
-  // warpgroups and merged in the CTA (needs at least two key tiles: more than 128 rows).  Non-causal dense
-  // items all cost the same: when their count leaves a last wave at most half full, those last items are
-  // split, so the last wave takes about half an item's time.  At d = 64, launches too small to fill the
-  // GPU split every item: non-causal ones with at most half as many items as SMs, causal ones (whose
-  // heaviest item sets the time of a single partial wave) with no more items than SMs.  (At d = 128 a split
-  // item streams twice the K/V bytes per key step -- its tiles serve one warpgroup each -- and measured
-  // no faster there.)  Packed (varlen) launches follow the same rules on their item count.
-  long long n_whole = n_items;
-  const int rows = (mode == eta::MODE_DENSE) ? N : max_len;
-  if (mode != eta::MODE_HSTU && d <= 128 && rows > 128) {
-    if (causal == 0 && n_items > G) {
-      const long long R = n_items % G;
-      if (R > 0 && 2 * R <= G) n_whole = n_items - R;
-    } else if (d == 64 && ((causal == 0 && 2 * n_items <= sms) || (causal != 0 && n_items <= sms))) {
-      n_whole = 0;
-    }
-  }
-  p.n_whole = (int)n_whole;
-  p.n_items = (int)(n_whole + 2 * (n_items - n_whole));
-  // persistent: at most one CTA per SM, and no more CTAs than (split) items
-  const dim3 grid((unsigned)std::min<long long>(p.n_items, sms), 1, 1);
+  if ((rc = plan_prefill(mode, units, rows, d, causal, sms, &pl)) != ETA_OK) return rc;
+  p.nblk = (int)pl.nblk;
+  p.n_whole = (int)pl.whole;
+  p.n_items = (int)pl.split_items;
+  const dim3 grid((unsigned)pl.ctas, 1, 1);
   p.sched_slot = next_sched_slot();
   p.o = o;
   p.lse = (mode == eta::MODE_HSTU) ? nullptr : lse;
@@ -489,6 +506,19 @@ int eta_selftest_wait_timeout(void *stream) {
   if (rc != ETA_OK) return rc;
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_wait_ns);
   return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
+}
+
+int eta_prefill_plan(int kind, long long units, long long rows, int d, int causal, int sms, long long *items,
+                     long long *whole, int *ctas) {
+  if (kind < eta::MODE_DENSE || kind > eta::MODE_HSTU) return ETA_ERR_ARG;
+  if (kind == eta::MODE_HSTU) causal = 1;
+  PrefillPlan pl;
+  const int rc = plan_prefill(kind, units, rows, d, causal, sms, &pl);
+  if (rc != ETA_OK) return rc;
+  if (items) *items = pl.items;
+  if (whole) *whole = pl.whole;
+  if (ctas) *ctas = pl.ctas;
+  return ETA_OK;
 }
 
 }  // extern "C"

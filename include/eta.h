@@ -214,6 +214,21 @@ ETA_API int attn_decode_noalloc(const void *q, const void *kcache, const void *v
                                 float *lse, int B, int H, int Lmax, int d, float scale, void *stream);
 
 /*
+ * eta_prefill_plan -- the work decomposition a prefill call would launch on a GPU with `sms` SMs (host
+ * logic only: no GPU is touched).  kind: 0 = attn_fwd / attn_fwd_fp8, 1 = attn_fwd_varlen,
+ * 2 = hstu_fwd_jagged (always causal).  units = B*H (dense) or S*H (packed); rows = N (dense) or max_len.
+ * A work item is 256 query rows (two 128-row Q tiles; 128 rows at d = 256) of one unit.  Outputs (each may be
+ * NULL): *items = work items; *whole = items run whole, the other items - whole are each run as two split
+ * halves (one Q tile, its key tiles divided between the CTA's two softmax warpgroups); *ctas = CTAs of the
+ * persistent grid.  The split rule: non-causal launches whose last wave is at most half full split those
+ * last items; at d = 64, causal launches with no more items than SMs and non-causal ones with at most half
+ * as many split every item; HSTU and d = 256 never split.
+ * Returns 0, or ETA_ERR_HEAD_DIM / ETA_ERR_SHAPE / ETA_ERR_ARG as the planned call would.
+ */
+ETA_API int eta_prefill_plan(int kind, long long units, long long rows, int d, int causal, int sms,
+                             long long *items, long long *whole, int *ctas);
+
+/*
  * eta_status -- synchronises `stream`, returns the device status word of the current device
  * (ETA_DEV_*; the first condition recorded since the last call) and clears it.  Returns ETA_ERR_CUDA if
  * the synchronisation or the copy failed.

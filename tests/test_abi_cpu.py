@@ -122,3 +122,35 @@ def test_fp8_host_validation(L):
     assert L.attn_fwd_fp8(A, A, A, A, NUL, 1, 1, 128, 128, 0.088, 1.0, 1.0, float("inf"), 0, 0, S) == -7
     assert L.attn_fwd_fp8(A, MIS, A, A, NUL, 1, 1, 128, 128, 0.088, 1.0, 1.0, 1.0, 0, 0, S) == -4
     assert L.attn_fwd_fp8(A, A, A, A, NUL, 1, 1, 128, 128, 0.088, 1.0, 1.0, 1.0, 0, 0, S) in (-6, -8)
+
+
+def test_prefill_plan_split_policy():
+    """The host's work decomposition (the same function the launches use), for a 148-SM B200."""
+    P = lambda *a: eta.prefill_plan(*a, sms=148)
+    # headline: 32 heads x 16 items of 256 rows; non-causal last wave 512 % 148 = 68 <= 74 -> 68 split
+    assert P("dense", 32, 4096, 64, False) == (512, 444, 148)
+    assert P("dense", 32, 4096, 64, True) == (512, 512, 148)   # causal, several waves: whole
+    # d = 64 launches too small to fill the GPU: every item split, one CTA per half
+    assert P("dense", 8, 2048, 64, True) == (64, 0, 128)
+    assert P("dense", 8, 2048, 64, False) == (64, 0, 128)
+    assert P("dense", 32, 1024, 64, True) == (128, 0, 148)
+    assert P("dense", 32, 1024, 64, False) == (128, 128, 128)  # 2 x 128 > 148: whole
+    # d = 128 keeps small launches whole; the non-causal last-wave rule still applies
+    assert P("dense", 32, 1024, 128, True) == (128, 128, 128)
+    assert P("dense", 20, 2000, 128, False) == (160, 148, 148)  # 160 % 148 = 12 split
+    assert P("dense", 148, 4096, 128, False) == (2368, 2368, 148)  # whole waves only
+    # one key tile per row block: nothing to split
+    assert P("dense", 8, 128, 64, True) == (8, 8, 8)
+    # HSTU never splits (and is always causal); d = 256 items are 128 rows, never split
+    assert P("hstu", 64, 4096, 64, False) == (1024, 1024, 148)
+    assert P("hstu", 4, 1024, 64, True) == (16, 16, 16)
+    assert P("dense", 64, 4096, 256, True) == (2048, 2048, 148)
+    # packed launches plan on S*H units of max_len rows
+    assert P("varlen", 30, 300, 64, True) == (60, 0, 120)
+    # rejected like the calls
+    with pytest.raises(eta.EtaError):
+        P("dense", 1, 128, 80, False)
+    with pytest.raises(eta.EtaError):
+        P("hstu", 1, 128, 256, True)
+    with pytest.raises(eta.EtaError):
+        P("dense", 0, 128, 64, False)
