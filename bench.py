@@ -7,8 +7,10 @@ A step is one pass of the hot path over the headline workload: prefill MHA with 
 TFLOP/s with the 4 n^2 d convention (halved for causal) over the whole job; L2 is flushed (a 256 MiB
 write) before every timed step, outside the timed events.  The same JSON line carries the roofline of the
 prefill kernel, an end-to-end number through the public API with host buffers, the oracle timed on the
-host cores, the SM clocks seen during timing, and (unless --no-extra) the other workloads of the method:
-prefill d=128 (B=8, causal) and its N sweep, HSTU over jagged sequences, and the decode step (GB/s).
+host cores, the SM clocks seen during timing, and (unless --no-extra) the other workloads of the method,
+each with the clocks seen while it ran: prefill d=128 (B=8, causal) and its N sweep, HSTU over jagged and
+dense sequences, head dims 96 and 256, e4m3 inputs, and the decode steps over a contiguous and a paged
+cache (GB/s).
 
 --impl reference times the fp64 CPU oracle (the only reference implementation this method has) on the
 same workload and metric, each step a bounded sample of it.
