@@ -7,8 +7,8 @@
 //
 // Design (B200):
 //  * grid (split, h, b); split i owns cache rows [i*chunk, min((i+1)*chunk, L_b)).  Splits past L_b exit.
-//  * one producer thread streams the split's K and V rows with 1-D bulk copies (cp.async.bulk, no
-//    multicast) into a DEC_STAGES-deep shared-memory ring of DEC_ROWS-row stages; each stage's K and V
+//  * one producer thread streams the split's K and V rows with 1-D bulk copies (cp.async.bulk) into
+//    a DEC_STAGES-deep shared-memory ring of DEC_ROWS-row stages; each stage's K and V
 //    rows are contiguous in HBM because the cache is [B, H, Lmax, d].
 //  * eight consumer warps take 4 rows of each stage; lane l holds d/32 consecutive elements of q, k and v,
 //    so a row's dot product is d/32 FMAs per lane plus a 5-step xor-shuffle reduction.  Each warp keeps

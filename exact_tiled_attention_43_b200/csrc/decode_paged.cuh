@@ -13,7 +13,7 @@
 //  * grid (split, kv head, b): split i owns cache rows [i*chunk, min((i+1)*chunk, L_b)) of sequence b; the
 //    CTA serves the G query heads of one KV head, so every K/V byte is read once for all G of them.
 //  * one producer thread reads the split's page numbers, then streams 32-row K and V stages with TMA
-//    (3-D tensor map over [page * Hkv + kv head, row in page, d], 128-byte swizzle, no multicast) through a
+//    (3-D tensor map over [page * Hkv + kv head, row in page, d], 128-byte swizzle) through a
 //    4-deep ring.  A stage is one 32-row slice of a page, or two 16-row pages.
 //  * two consumer warps take alternate stages.  The G queries (padded to 16 rows) stay in registers as
 //    warp-MMA A fragments; S = Q K^T, the online softmax and O += P V run on 16 x 32 register tiles

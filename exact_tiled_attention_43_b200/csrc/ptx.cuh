@@ -1,5 +1,5 @@
 // ptx.cuh -- thin inline-PTX wrappers for the sm_100a features the kernels use: mbarriers with bounded
-// waits, TMA tensor/bulk copies (never with cluster multicast), and tcgen05 (TMEM allocation, MMA issue,
+// waits, TMA tensor/bulk copies (each CTA loads its own copy), and tcgen05 (TMEM allocation, MMA issue,
 // commit, TMEM loads/stores, fences).  Each wrapper is one documented PTX instruction.
 #pragma once
 
