@@ -205,6 +205,19 @@ def test_library_cross_check_tiny_config():
         np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), atol=1e-12)
 
 
+@pytest.mark.parametrize("d", [96, 128, 256])
+def test_library_cross_check_other_head_dims(d):
+    # The head dims the kernels also serve, against torch's fp64 CPU scaled_dot_product_attention (a ragged
+    # length, so that no tile boundary is special).
+    q, k, v = (inputs.normal_bf16((1, 2, 150, d), 95 + i, 1.0) for i in range(3))
+    scale = float(np.float32(1 / math.sqrt(d)))
+    for causal in (False, True):
+        o, lse = oracle.attn(q, k, v, scale, causal)
+        ref = torch.nn.functional.scaled_dot_product_attention(q.double(), k.double(), v.double(),
+                                                                is_causal=causal, scale=scale)
+        np.testing.assert_allclose(o, ref.numpy(), atol=1e-12)
+
+
 def test_sampled_rows_match_full():
     B, H, N, d = 1, 3, 70, 8
     q, k, v = (_rand((B, H, N, d), 90 + i) for i in range(3))
