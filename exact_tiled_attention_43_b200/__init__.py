@@ -119,6 +119,33 @@ def _need(t, name, dtype, ndim):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _same_device(ref, *tensors):
+    for name, t in tensors:
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, expected {ref.device} (all tensors of a call on one GPU)")
+
+
+def _check_buf(t, name, shape, dtypes, device):
+    """A caller-provided output or workspace: the kernels write exactly `shape` elements of one of `dtypes`
+    through its pointer, so anything else is refused before a launch could write past it."""
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must be one of {dtypes}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _device_ctx(t):
+    """Makes t's GPU current for the call, so that the library and the default stream are t's."""
+    return _torch().cuda.device(t.device)
+
+
 def default_scale(d: int) -> float:
     """The float32 value of 1/sqrt(d)."""
     import numpy as np
@@ -135,15 +162,20 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out_dtyp
     B, H, N, d = q.shape
     if k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v must have the same shape")
+    _same_device(q, ("k", k), ("v", v))
     out_dtype = out_dtype or torch.bfloat16
     if out is None:
         out = torch.empty((B, H, N, d), dtype=out_dtype, device=q.device)
+    _check_buf(out, "out", (B, H, N, d), (torch.bfloat16, torch.float32), q.device)
     if return_lse and lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if return_lse:
+        _check_buf(lse, "lse", (B, H, N), (torch.float32,), q.device)
     scale = default_scale(d) if scale is None else float(scale)
     odt = ETA_OUT_F32 if out.dtype == torch.float32 else ETA_OUT_BF16
-    rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse if return_lse else None), B, H, N, d, scale,
-                        int(bool(causal)), odt, _stream_ptr(stream))
+    with _device_ctx(q):
+        rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse if return_lse else None), B, H, N, d,
+                            scale, int(bool(causal)), odt, _stream_ptr(stream))
     _check(rc, "attn_fwd")
     return out, (lse if return_lse else None)
 
@@ -159,16 +191,22 @@ def attn_fwd_fp8(q8, k8, v8, q_descale: float, k_descale: float, v_descale: floa
     if k8.shape != q8.shape or v8.shape != q8.shape:
         raise ValueError("q8, k8, v8 must have the same shape")
     B, H, N, d = q8.shape
-    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
-    odt = {torch.bfloat16: 0, torch.float32: 1}[out_dtype]
+    _same_device(q8, ("k8", k8), ("v8", v8))
     if out is None:
-        out = torch.empty((B, H, N, d), dtype=out_dtype, device=q8.device)
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16 if out_dtype is None else out_dtype, device=q8.device)
+    _check_buf(out, "out", (B, H, N, d), (torch.bfloat16, torch.float32), q8.device)
+    odt = ETA_OUT_F32 if out.dtype == torch.float32 else ETA_OUT_BF16
     if lse is None and return_lse:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    if not return_lse:
+        lse = None
+    if lse is not None:
+        _check_buf(lse, "lse", (B, H, N), (torch.float32,), q8.device)
     scale = default_scale(d) if scale is None else float(scale)
-    rc = lib().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(out), _ptr(lse) if lse is not None else None, B, H, N,
-                            d, scale, float(q_descale), float(k_descale), float(v_descale), int(bool(causal)), odt,
-                            _stream_ptr(stream))
+    with _device_ctx(q8):
+        rc = lib().attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(out), _ptr(lse), B, H, N, d, scale,
+                                float(q_descale), float(k_descale), float(v_descale), int(bool(causal)), odt,
+                                _stream_ptr(stream))
     _check(rc, "attn_fwd_fp8")
     return out, lse
 
@@ -182,13 +220,17 @@ def attn_fwd_varlen(q, k, v, cu_seqlens, max_len: int, causal: bool = False, sca
         _need(t, n, torch.bfloat16, 3)
     _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
     T, H, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape")
+    _same_device(q, ("k", k), ("v", v), ("cu_seqlens", cu_seqlens))
     out = torch.empty((T, H, d), dtype=out_dtype or torch.bfloat16, device=q.device)
     lse = torch.empty((T, H), dtype=torch.float32, device=q.device) if return_lse else None
     scale = default_scale(d) if scale is None else float(scale)
     odt = ETA_OUT_F32 if out.dtype == torch.float32 else ETA_OUT_BF16
-    rc = lib().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens),
-                               cu_seqlens.numel() - 1, int(max_len), T, H, d, scale, int(bool(causal)), odt,
-                               _stream_ptr(stream))
+    with _device_ctx(q):
+        rc = lib().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens),
+                                   cu_seqlens.numel() - 1, int(max_len), T, H, d, scale, int(bool(causal)), odt,
+                                   _stream_ptr(stream))
     _check(rc, "attn_fwd_varlen")
     return out, lse
 
@@ -200,10 +242,15 @@ def hstu_fwd_jagged(q, k, v, cu_seqlens, max_len: int, alpha: float, inv_n: floa
         _need(t, n, torch.bfloat16, 3)
     _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
     T, H, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape")
+    _same_device(q, ("k", k), ("v", v), ("cu_seqlens", cu_seqlens))
     if out is None:
         out = torch.empty((T, H, d), dtype=torch.bfloat16, device=q.device)
-    rc = lib().hstu_fwd_jagged(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
-                               int(max_len), T, H, d, float(alpha), float(inv_n), _stream_ptr(stream))
+    _check_buf(out, "out", (T, H, d), (torch.bfloat16,), q.device)
+    with _device_ctx(q):
+        rc = lib().hstu_fwd_jagged(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                                   int(max_len), T, H, d, float(alpha), float(inv_n), _stream_ptr(stream))
     _check(rc, "hstu_fwd_jagged")
     return out
 
@@ -224,16 +271,22 @@ def attn_decode(q, kcache, vcache, kv_lens, scale: float | None = None, workspac
     B, H, Lmax, d = kcache.shape
     if vcache.shape != kcache.shape or q.shape != (B, H, d) or kv_lens.shape != (B,):
         raise ValueError("inconsistent decode shapes")
+    _same_device(q, ("kcache", kcache), ("vcache", vcache), ("kv_lens", kv_lens))
     need = attn_decode_workspace_size(B, H, Lmax, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check_buf(workspace, "workspace", None, (workspace.dtype,), q.device)
     if out is None:
         out = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
+    _check_buf(out, "out", (B, H, d), (torch.bfloat16,), q.device)
     if lse is None:
         lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    _check_buf(lse, "lse", (B, H), (torch.float32,), q.device)
     scale = default_scale(d) if scale is None else float(scale)
-    rc = lib().attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kv_lens), _ptr(out), _ptr(lse), B, H, Lmax, d,
-                           scale, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    with _device_ctx(q):
+        rc = lib().attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kv_lens), _ptr(out), _ptr(lse), B, H, Lmax,
+                               d, scale, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream_ptr(stream))
     _check(rc, "attn_decode")
     return out, lse
 
@@ -258,17 +311,23 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, kv_lens, scale: float | 
     max_pages = block_table.shape[1]
     if v_pages.shape != k_pages.shape or dq != d or block_table.shape[0] != B or kv_lens.shape != (B,):
         raise ValueError("inconsistent paged decode shapes")
+    _same_device(q, ("k_pages", k_pages), ("v_pages", v_pages), ("block_table", block_table), ("kv_lens", kv_lens))
     need = attn_decode_paged_workspace_size(B, Hq, max_pages, page_size, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check_buf(workspace, "workspace", None, (workspace.dtype,), q.device)
     if out is None:
         out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    _check_buf(out, "out", (B, Hq, d), (torch.bfloat16,), q.device)
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check_buf(lse, "lse", (B, Hq), (torch.float32,), q.device)
     scale = default_scale(d) if scale is None else float(scale)
-    rc = lib().attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(kv_lens), _ptr(out),
-                                 _ptr(lse), B, Hq, Hkv, num_pages, page_size, max_pages, d, scale, _ptr(workspace),
-                                 workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    with _device_ctx(q):
+        rc = lib().attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(kv_lens),
+                                     _ptr(out), _ptr(lse), B, Hq, Hkv, num_pages, page_size, max_pages, d, scale,
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream_ptr(stream))
     _check(rc, "attn_decode_paged")
     return out, lse
 
@@ -288,13 +347,17 @@ def attn_decode_noalloc(q, kcache, vcache, kv_lens, scale: float | None = None, 
     B, H, Lmax, d = kcache.shape
     if vcache.shape != kcache.shape or q.shape != (B, H, d) or kv_lens.shape != (B,):
         raise ValueError("inconsistent decode shapes")
+    _same_device(q, ("kcache", kcache), ("vcache", vcache), ("kv_lens", kv_lens))
     if out is None:
         out = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
+    _check_buf(out, "out", (B, H, d), (torch.bfloat16,), q.device)
     if lse is None:
         lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    _check_buf(lse, "lse", (B, H), (torch.float32,), q.device)
     scale = default_scale(d) if scale is None else float(scale)
-    rc = lib().attn_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kv_lens), _ptr(out), _ptr(lse), B, H,
-                                   Lmax, d, scale, _stream_ptr(stream))
+    with _device_ctx(q):
+        rc = lib().attn_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kv_lens), _ptr(out), _ptr(lse), B,
+                                       H, Lmax, d, scale, _stream_ptr(stream))
     _check(rc, "attn_decode_noalloc")
     return out, lse
 
