@@ -154,3 +154,22 @@ def test_prefill_plan_split_policy():
         P("hstu", 1, 128, 256, True)
     with pytest.raises(eta.EtaError):
         P("dense", 0, 128, 64, False)
+
+
+def test_header_is_c99_and_library_links_from_c(tmp_path):
+    """The public header compiles as strict C99 and a C program links against libeta.so and gets answers
+    from the host-side entry points (no GPU is used)."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lib_dir = os.path.dirname(eta.LIB_PATH)
+    exe = str(tmp_path / "abi_c_check")
+    subprocess.check_call([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                           "-I", os.path.join(root, "include"), os.path.join(root, "tests", "abi_c_check.c"),
+                           "-o", exe, "-L", lib_dir, "-leta", "-Wl,-rpath," + lib_dir])
+    out = subprocess.run([exe], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)
