@@ -147,6 +147,12 @@ def test_prefill_plan_split_policy():
     assert P("dense", 64, 4096, 256, True) == (2048, 2048, 148)
     # packed launches plan on S*H units of max_len rows
     assert P("varlen", 30, 300, 64, True) == (60, 0, 120)
+    # size limits: a row-block count past 65535, an item count past the work counter's range
+    assert P("dense", 1, 256 * 65535, 64, False)[0] == 65535
+    with pytest.raises(eta.EtaError):
+        P("dense", 1, 256 * 65535 + 1, 64, False)
+    with pytest.raises(eta.EtaError):
+        P("dense", 2 ** 31 // 4, 4096, 64, False)
     # rejected like the calls
     with pytest.raises(eta.EtaError):
         P("dense", 1, 128, 80, False)
