@@ -61,3 +61,27 @@ def test_single_process_defaults():
     assert not ctx.on and ctx.max(3.5) == 3.5
     assert bench.attn_flops(1, 32, 4096, 64, False) == 2 * bench.attn_flops(1, 32, 4096, 64, True)
     assert bench.attn_flops(1, 32, 4096, 64, False) == 4 * 32 * 4096 ** 2 * 64
+
+
+def test_kernel_source_hash_ignores_comments(tmp_path, monkeypatch):
+    """Recorded profiler counters stay keyed to the kernel code: a comment-only edit keeps the hash, a code
+    edit changes it."""
+    import shutil
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    csrc = tmp_path / "exact_tiled_attention_43_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in ("ptx.cuh", "prefill.cuh", "decode.cuh"):
+        shutil.copy(os.path.join(ROOT, "exact_tiled_attention_43_b200", "csrc", f), csrc / f)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash()
+    assert h0 == bench.__dict__["kernel_source_hash"]()
+    p = csrc / "prefill.cuh"
+    src = p.read_text()
+    p.write_text("// a new comment line\n" + src.replace("#pragma once", "#pragma once  // trailing note /* x */", 1))
+    assert bench.kernel_source_hash() == h0
+    p.write_text(src + "\nstatic const int eta_extra_constant = 1;\n")
+    assert bench.kernel_source_hash() != h0
