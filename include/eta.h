@@ -97,7 +97,9 @@ ETA_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float
  *   o          : [T, H, d] bf16 or fp32 (o_dtype);  lse: fp32 [T, H] or NULL
  *   cu_seqlens : int32 [S+1], device; cu_seqlens[0] = 0, non-decreasing
  *   max_len    : an upper bound on every sequence length (sizes the launch); T_total : cu_seqlens[S]
- *                as known to the host (used to size tensor maps; must match the device value)
+ *                as known to the host (used to size tensor maps; must match the device value: the
+ *                kernels check that offsets do not decrease and that no sequence exceeds max_len, not
+ *                that the last offset stays within T_total, so a larger value would write rows past o)
  *   No query attends across a sequence boundary; causal is per sequence (local indices).
  * Zero-length sequences produce nothing.  Errors as attn_fwd, plus device status ETA_DEV_BAD_CUSEQ.
  */
@@ -197,7 +199,7 @@ ETA_API int attn_decode_paged(const void *q, const void *k_pages, const void *v_
  * allocation in its enqueue step, or a latency-critical loop that cannot afford cudaMalloc's implicit
  * device synchronisation.  It takes no workspace argument: the split-KV partial results go to a fixed
  * scratch array of ETA_NOALLOC_SCRATCH_BYTES that the library holds in device memory (one copy on every GPU
- * that loads the library, kept until the process exits).  The paper has no counterpart; it is an
+ * that loads the library, kept until the process exits).  The pages have no counterpart; it is an
  * interface convenience around the decode kernels.
  *   Arguments, layouts and results are exactly those of attn_decode (minus workspace / workspace_bytes).
  *   The first call on a device, with that device current, looks up the scratch array's device address
