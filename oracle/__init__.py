@@ -18,15 +18,39 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
-_LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 
+def _host_tag() -> str:
+    """A short tag of this host's CPU (model and feature flags).  The library is built for the host it runs on
+    (-march=native), so a copy built on another machine is never loaded here."""
+    import hashlib
+    import platform
+
+    ident = platform.machine()
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith(("model name", "flags", "Features", "CPU part")):
+                    ident += line
+                    if line.startswith(("flags", "Features")):
+                        break
+    except OSError:
+        pass
+    return hashlib.sha256(ident.encode()).hexdigest()[:12]
+
+
+_LIB = os.path.join(_HERE, f"liboracle-{_host_tag()}.so")
+
+
 def build(force: bool = False) -> str:
-    """Compile oracle.c into liboracle.so (gcc, -O2, OpenMP, strict IEEE: no -ffast-math)."""
+    """Compile oracle.c into a library for this host (gcc -O3 -march=native, OpenMP).  The arithmetic stays
+    strict IEEE double in source order: no -ffast-math, and -ffp-contract=off so that no multiply-add is
+    fused, which makes the results identical to any other conforming build."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + ".tmp.%d" % os.getpid()
-        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        subprocess.check_call(["gcc", "-O3", "-march=native", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
+                               "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -51,6 +75,8 @@ def _load():
         lib.oracle_decode_paged.argtypes = [dp, dp, dp, ip, ip, i, i, i, i, i, i, ctypes.c_double, dp, dp]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
+        lib.oracle_set_num_threads.restype = None
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -90,6 +116,11 @@ def _ip(a):
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of later calls (n <= 0: the OpenMP default).  Timing only; results do not depend on it."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def attn(q, k, v, scale: float, causal: bool, rows=None, return_flops: bool = False):

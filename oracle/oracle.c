@@ -211,6 +211,18 @@ EXPORT int64_t oracle_decode_paged(const double *q, const double *k_pages, const
     return 2 * macs;
 }
 
+/* Threads later oracle calls use (the timed CPU baseline reports a one-core figure as well); n <= 0
+ * leaves the OpenMP default.  Touches no arithmetic. */
+EXPORT void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* Number of OpenMP threads the oracle will use (reported with timed CPU baselines). */
 EXPORT int oracle_num_threads(void)
 {
