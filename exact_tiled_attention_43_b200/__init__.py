@@ -43,6 +43,7 @@ SIGNATURES = {
     "eta_selftest_wait_timeout": (_I, [_VP]),
     "eta_prefill_plan": (_I, [_I, _LL, _LL, _I, _I, _I, ctypes.POINTER(ctypes.c_longlong),
                               ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_int)]),
+    "eta_prefill_sched_group": (_LL, [_LL, _LL, _I, _I]),
 }
 
 
@@ -78,6 +79,14 @@ def prefill_plan(kind: str, units: int, rows: int, d: int, causal: bool, sms: in
                                 ctypes.byref(items), ctypes.byref(whole), ctypes.byref(ctas))
     _check(rc, "eta_prefill_plan")
     return items.value, whole.value, ctas.value
+
+
+def prefill_sched_group(units: int, rows: int, d: int, elt_bytes: int = 2) -> int:
+    """(batch, head) units a dense prefill launch schedules together so that their K/V stay in L2 (host logic,
+    no GPU)."""
+    g = int(lib().eta_prefill_sched_group(int(units), int(rows), int(d), int(elt_bytes)))
+    _check(g if g < 0 else 0, "eta_prefill_sched_group")
+    return g
 
 
 def strerror(code: int) -> str:

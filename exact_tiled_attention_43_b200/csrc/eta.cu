@@ -157,6 +157,16 @@ struct PrefillPlan {
   long long nblk = 0, items = 0, whole = 0, split_items = 0;
   int ctas = 0;
 };
+
+// Dense launches take their (batch, head) units in groups whose K and V (2 * rows * d * elt bytes per unit)
+// fit in this many bytes, a quarter of the B200's L2, so that the row blocks of a unit find its K/V tiles
+// in L2 (the kernels' decode_item order).
+constexpr long long kSchedGroupBytes = 32ll << 20;
+long long sched_group(long long units, long long rows, int d, int elt) {
+  const long long kv = 2 * rows * (long long)d * elt;
+  const long long g = kv > 0 ? kSchedGroupBytes / kv : units;
+  return std::max<long long>(1, std::min<long long>(g, units));
+}
 int plan_prefill(int mode, long long units, long long rows, int d, int causal, int sms, PrefillPlan *pl) {
   if (d != 64 && d != 96 && d != 128 && !(d == 256 && mode != eta::MODE_HSTU)) return ETA_ERR_HEAD_DIM;
   if (units <= 0 || rows <= 0 || sms <= 0) return ETA_ERR_SHAPE;
@@ -217,6 +227,7 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
     n2 = units;
     p.N = N;
     p.BH = (int)units;
+    p.grp = (int)sched_group(units, rows, d, f8 ? 1 : 2);
   } else {
     if (S <= 0 || max_len <= 0 || T_total < 0 || S > 65535) return ETA_ERR_SHAPE;
     if (T_total == 0) return ETA_OK;  // nothing to compute
@@ -226,6 +237,7 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
     n2 = T_total;
     p.max_len = max_len;
     p.S = S;
+    p.T_total = T_total;
   }
   if (mode == eta::MODE_HSTU) {
     if (!std::isfinite(alpha) || !finite_pos(inv_n)) return ETA_ERR_ARG;
@@ -484,7 +496,9 @@ const char *eta_strerror(int code) {
   switch (code) {
     case ETA_OK: return "ok";
     case ETA_ERR_NULL: return "a required pointer is NULL";
-    case ETA_ERR_HEAD_DIM: return "unsupported head dimension (64, 128; 256 for attn_fwd / attn_fwd_varlen)";
+    case ETA_ERR_HEAD_DIM:
+      return "unsupported head dimension (attn_fwd, attn_fwd_varlen: 64, 96, 128, 256; hstu_fwd_jagged: 64, 96, 128; "
+             "attn_fwd_fp8: 128; attn_decode, attn_decode_paged: 64, 128)";
     case ETA_ERR_SHAPE: return "a size is out of range or inconsistent";
     case ETA_ERR_ALIGN: return "a tensor pointer is not 16-byte aligned";
     case ETA_ERR_WORKSPACE: return "workspace is smaller than attn_decode_workspace_size()";
@@ -493,7 +507,9 @@ const char *eta_strerror(int code) {
     case ETA_ERR_DEVICE: return "the current device is not an sm_100 GPU";
     case ETA_DEV_TIMEOUT: return "device: a bounded pipeline wait expired";
     case ETA_DEV_BAD_KVLEN: return "device: kv_lens entry outside [0, Lmax]";
-    case ETA_DEV_BAD_CUSEQ: return "device: cu_seqlens decreasing or a sequence longer than max_len";
+    case ETA_DEV_BAD_CUSEQ:
+      return "device: cu_seqlens not a valid offset table for the call (negative or decreasing, a sequence longer "
+             "than max_len, first offset not 0 or last offset not T_total)";
     case ETA_DEV_BAD_PAGE: return "device: a block_table entry outside [0, num_pages)";
     default: return "unknown code";
   }
@@ -506,6 +522,11 @@ int eta_selftest_wait_timeout(void *stream) {
   if (rc != ETA_OK) return rc;
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_wait_ns);
   return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
+}
+
+long long eta_prefill_sched_group(long long units, long long rows, int d, int elt_bytes) {
+  if (units <= 0 || rows <= 0 || d <= 0 || (elt_bytes != 1 && elt_bytes != 2)) return ETA_ERR_SHAPE;
+  return sched_group(units, rows, d, elt_bytes);
 }
 
 int eta_prefill_plan(int kind, long long units, long long rows, int d, int causal, int sms, long long *items,

@@ -88,6 +88,8 @@ struct PrefillParams {
   const int *cu_seqlens;   // packed modes: [S+1]
   int H, N, max_len;       // N: dense sequence length
   int BH, S;               // dense: B*H; packed: number of sequences
+  int T_total;             // packed: rows of q/k/v/o (the last offset the host was given)
+  int grp;                 // dense: (batch, head) units per scheduling group (see decode_item)
   int nblk;                // 256-row blocks per (batch|sequence, head)
   int n_items;             // work indices: n_whole whole items, then two split halves per remaining item
   int n_whole;             // items (in heaviest-first order) processed whole; the rest are split
@@ -220,7 +222,37 @@ struct PfSmem {
   }
 };
 
-// Work item `idx`, heaviest first: the latest row block of every (batch|sequence, head) comes first.
+// Sequence s of a packed launch: its first row and length, checked against the launch's contract.  A
+// sequence whose rows would leave [0, T_total) (a negative or decreasing offset, a length above max_len, an
+// end past T_total) gets length 0 and is skipped, so no load or store of it happens; every breach of the
+// contract (also a first offset other than 0 or a last one other than T_total, which stay in bounds) records
+// ETA_DEV_BAD_CUSEQ once, from the sequence's block-0, head-0 item.
+__device__ __forceinline__ void packed_sequence(const PrefillParams &p, int s, bool report, int &start, int &L) {
+  const int a = p.cu_seqlens[s], b = p.cu_seqlens[s + 1];
+  const bool unsafe = a < 0 || b < a || b - a > p.max_len || b > p.T_total;
+  const bool off_contract = (s == 0 && a != 0) || (s == p.S - 1 && b != p.T_total);
+  if ((unsafe || off_contract) && report) record_status(3 /* ETA_DEV_BAD_CUSEQ */);
+  start = unsafe ? 0 : a;
+  L = unsafe ? 0 : b - a;
+}
+
+// Dense work item `idx` -> (unit, row block).  Units ((batch, head) pairs) are taken in groups of p.grp,
+// sized on the host so that one group's K and V stay resident in L2; inside a group the latest (heaviest,
+// when causal) row block of every unit comes first.  The K/V tiles of a unit are then read from HBM about
+// once, shared through L2 by its row blocks, instead of once per row block when all units run each level
+// together.  The last group's light blocks still end the launch (heaviest-first tail).
+__device__ __forceinline__ void dense_unit_block(const PrefillParams &p, int idx, int &unit, int &blk) {
+  const int per_grp = p.grp * p.nblk;
+  const int g = idx / per_grp;
+  const int u0 = g * p.grp;
+  const int gsz = min(p.grp, p.BH - u0);
+  const int rem = idx - g * per_grp;
+  blk = p.nblk - 1 - rem / gsz;
+  unit = u0 + (rem - (rem / gsz) * gsz);
+}
+
+// Work item `idx`: packed launches take the latest row block of every (sequence, head) first; dense ones go
+// group by group (dense_unit_block).
 template <int D, int MODE>
 __device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int idx) {
   constexpr int BN = PfCfg<D>::BN;
@@ -237,15 +269,9 @@ __device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int idx) {
     const int rem = idx - (idx / per) * per;
     const int s = rem / p.H;
     it.h = rem - s * p.H;
-    it.seq_start = p.cu_seqlens[s];
-    it.L = p.cu_seqlens[s + 1] - it.seq_start;
-    if (it.L < 0 || it.L > p.max_len) {
-      if (blk == 0 && it.h == 0) record_status(3 /* ETA_DEV_BAD_CUSEQ */);
-      it.L = 0;  // the sequence is skipped
-    }
+    packed_sequence(p, s, blk == 0 && it.h == 0, it.seq_start, it.L);
   } else {
-    blk = p.nblk - 1 - idx / p.BH;
-    it.bh = idx - (idx / p.BH) * p.BH;
+    dense_unit_block(p, idx, it.bh, blk);
     it.L = p.N;
   }
   it.r0 = blk * 2 * PF_BM;

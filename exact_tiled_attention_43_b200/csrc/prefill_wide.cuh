@@ -81,8 +81,9 @@ struct WideSmem {
   }
 };
 
-// Work item `idx` (heaviest first: the latest 128-row block of every (batch|sequence, head) comes first).
-// n0 = key tiles the block sees.
+// Work item `idx` (128-row blocks; packed: the latest block of every (sequence, head) first; dense: units
+// in L2-sized groups, heaviest block first inside a group -- the order of decode_item).  n0 = key tiles the
+// block sees.
 template <int MODE>
 __device__ __forceinline__ PfItem wide_decode_item(const PrefillParams &p, int idx) {
   PfItem it{};
@@ -93,15 +94,9 @@ __device__ __forceinline__ PfItem wide_decode_item(const PrefillParams &p, int i
     const int rem = idx - (idx / per) * per;
     const int s = rem / p.H;
     it.h = rem - s * p.H;
-    it.seq_start = p.cu_seqlens[s];
-    it.L = p.cu_seqlens[s + 1] - it.seq_start;
-    if (it.L < 0 || it.L > p.max_len) {
-      if (blk == 0 && it.h == 0) record_status(3 /* ETA_DEV_BAD_CUSEQ */);
-      it.L = 0;
-    }
+    packed_sequence(p, s, blk == 0 && it.h == 0, it.seq_start, it.L);
   } else {
-    blk = p.nblk - 1 - idx / p.BH;
-    it.bh = idx - (idx / p.BH) * p.BH;
+    dense_unit_block(p, idx, it.bh, blk);
     it.L = p.N;
   }
   it.r0 = blk * PF_BM;

@@ -28,8 +28,8 @@
  *    returns; results are ready when the stream reaches that point.
  *  - Return value: 0 (ETA_OK) when the work was enqueued, a negative ETA_ERR_* code when the arguments
  *    are rejected on the host (nothing is enqueued then) or a CUDA launch failed.
- *  - Conditions only the device can see (a kv_lens entry outside [0, Lmax], cu_seqlens that decrease or
- *    hold a sequence longer than max_len, a pipeline wait that ran out of time) never trap: the kernel
+ *  - Conditions only the device can see (a kv_lens entry outside [0, Lmax], a cu_seqlens table that is not
+ *    valid for the call, a pipeline wait that ran out of time) never trap: the kernel
  *    keeps every access in bounds, records the first such condition in a device status word and carries
  *    on or returns.  Read it with eta_status().
  *  - Head dimension d: 64, 96 or 128 for every prefill call, 256 for softmax attention (attn_fwd,
@@ -66,7 +66,7 @@ extern "C" {
 #define ETA_DEV_OK 0
 #define ETA_DEV_TIMEOUT 1     /* a bounded pipeline wait expired; the kernel abandoned its tile */
 #define ETA_DEV_BAD_KVLEN 2   /* attn_decode: kv_lens[b] < 0 or > Lmax (clamped into range) */
-#define ETA_DEV_BAD_CUSEQ 3   /* varlen/jagged: cu_seqlens decreasing or a sequence longer than max_len */
+#define ETA_DEV_BAD_CUSEQ 3   /* varlen/jagged: cu_seqlens not a valid offset table for the call (see attn_fwd_varlen) */
 #define ETA_DEV_BAD_PAGE 4    /* attn_decode_paged: a block_table entry outside [0, num_pages) (page 0 read) */
 
 /* Output element type selector for attn_fwd / attn_fwd_varlen. */
@@ -92,15 +92,32 @@ ETA_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float
              float scale, int causal, int o_dtype, void *stream);
 
 /*
+ * Launches in flight (every prefill call: attn_fwd, attn_fwd_varlen, attn_fwd_fp8, hstu_fwd_jagged).
+ * A prefill launch hands out its work items from a device counter.  The library holds 256 such counters per
+ * device and gives each launch the next one, round-robin, when the call enqueues it; the launch's last CTA
+ * returns the counter to zero.  So:
+ *   - at most 256 prefill launches may be in flight on one device at a time (enqueued and not finished,
+ *     over all streams); a 257th would share a counter with a launch still running, and both would skip or
+ *     repeat work items;
+ *   - a CUDA graph that captured a prefill call keeps that call's counter for good: do not replay one graph
+ *     on two streams at once, and do not keep a replay in flight while 256 other prefill launches are
+ *     enqueued after it.
+ * Launches ordered on one stream never overlap, so ordinary use needs nothing.
+ */
+
+/*
  * attn_fwd_varlen -- exact attention over S packed sequences (no padding).
  *   q, k, v    : bf16 [T, H, d], T = cu_seqlens[S]; sequence s owns rows cu_seqlens[s] .. cu_seqlens[s+1]-1
  *   o          : [T, H, d] bf16 or fp32 (o_dtype);  lse: fp32 [T, H] or NULL
  *   cu_seqlens : int32 [S+1], device; cu_seqlens[0] = 0, non-decreasing
  *   max_len    : an upper bound on every sequence length (sizes the launch); T_total : cu_seqlens[S]
- *                as known to the host (used to size tensor maps; must match the device value: the
- *                kernels check that offsets do not decrease and that no sequence exceeds max_len, not
- *                that the last offset stays within T_total, so a larger value would write rows past o)
+ *                as known to the host: the rows of q, k, v, o (and of lse) the call may touch
  *   No query attends across a sequence boundary; causal is per sequence (local indices).
+ * The kernels read cu_seqlens on the device and check it against the call ("同样是Attention架构..." page,
+ * section "绝杀优化三：Jagged变长张量": the offsets are the whole state of a jagged tensor).  A sequence whose
+ * offsets are negative or decreasing, longer than max_len, or end past T_total is skipped (nothing of it is
+ * read or written, so no access leaves [0, T_total)); that, and a first offset other than 0 or a last offset
+ * other than T_total (sequences inside [0, T_total) are still computed), record ETA_DEV_BAD_CUSEQ.
  * Zero-length sequences produce nothing.  Errors as attn_fwd, plus device status ETA_DEV_BAD_CUSEQ.
  */
 ETA_API int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse, const int *cu_seqlens,
@@ -229,6 +246,15 @@ ETA_API int attn_decode_noalloc(const void *q, const void *kcache, const void *v
  */
 ETA_API int eta_prefill_plan(int kind, long long units, long long rows, int d, int causal, int sms,
                              long long *items, long long *whole, int *ctas);
+
+/*
+ * eta_prefill_sched_group -- how many (batch, head) units a dense prefill launch (attn_fwd, attn_fwd_fp8)
+ * schedules together (host logic only).  Items are handed out group by group, and inside a group the latest
+ * row block of every unit first, so that the K and V of a group (2 * rows * d * elt_bytes bytes per unit,
+ * kept within 32 MiB) stay in L2 while its row blocks run and are read from HBM about once.  rows = N;
+ * elt_bytes = 2 (bf16) or 1 (e4m3).  Returns a count in [1, units], or ETA_ERR_SHAPE.
+ */
+ETA_API long long eta_prefill_sched_group(long long units, long long rows, int d, int elt_bytes);
 
 /*
  * eta_status -- synchronises `stream`, returns the device status word of the current device
