@@ -162,6 +162,23 @@ def test_prefill_plan_split_policy():
         P("dense", 0, 128, 64, False)
 
 
+def test_prefill_sched_group():
+    """Dense launches schedule their (batch, head) units in groups whose K and V (2 * N * d * elt bytes a
+    unit) fit in 32 MiB, at least one unit and at most all of them."""
+    G = eta.prefill_sched_group
+    assert G(32, 4096, 64) == 32        # B1 H32 N4096 d64: 1 MiB a unit, all 32 units in one group
+    assert G(256, 4096, 128) == 16      # B8 H32 N4096 d128: 2 MiB a unit
+    assert G(256, 4096, 128, 1) == 32   # the same shape in e4m3: 1 MiB a unit
+    assert G(64, 4096, 256) == 8        # d = 256: 4 MiB a unit
+    assert G(32, 32768, 128) == 2       # N = 32k: 16 MiB a unit
+    assert G(32, 65536, 256) == 1       # 64 MiB a unit: one unit per group
+    assert G(80, 2048, 128) == 32       # 1 MiB a unit, 80 units: groups of 32, 32, 16
+    assert G(5, 1000, 64) == 5          # fewer units than fit
+    for bad in ((0, 4096, 64, 2), (1, 0, 64, 2), (1, 4096, 64, 4)):
+        with pytest.raises(eta.EtaError):
+            G(*bad)
+
+
 def test_header_is_c99_and_library_links_from_c(tmp_path):
     """The public header compiles as strict C99 and a C program links against libeta.so and gets answers
     from the host-side entry points (no GPU is used)."""

@@ -88,3 +88,57 @@ def test_hstu_dense_page_shape_sampled(N):
         sub = lambda x: x[a:b, heads].contiguous()
         o_ref = oracle.hstu_jagged(sub(q), sub(k), sub(v), [0, N], 0.125, 1.0 / N)
         check_hstu(sub(o), o_ref, f"hstu dense N={N} seq={s}")
+
+
+def _vp(t):
+    import ctypes
+
+    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+SENTINEL = 7.0  # never an attention output here (|o| <= max |v| < 7 for these inputs, HSTU outputs ~1e-2)
+
+
+@pytest.mark.parametrize("kind,d", [("varlen", 64), ("varlen", 128), ("varlen", 256), ("hstu", 64), ("hstu", 96)])
+@pytest.mark.parametrize("tail", ["past_end", "short", "negative_start"])
+def test_cu_seqlens_checked_against_T_total(kind, d, tail):
+    """The packed kernels read cu_seqlens on the device and check it against the T_total the call was given.
+    The q/k/v/o/lse buffers hold T_total rows followed by 64 guard rows; the offset table is broken in one
+    of three ways:
+      past_end       : the last offset is 100 rows past T_total -> that sequence is skipped;
+      short          : the last offset is 60 rows short of T_total -> in bounds, every sequence computed;
+      negative_start : the first offset is -5 -> the first sequence is skipped.
+    Each records ETA_DEV_BAD_CUSEQ; every computed sequence matches the oracle; skipped sequences, rows past
+    the table's end and the guard rows keep their sentinel value."""
+    H, T, G = 2, 420, 64
+    bounds = {"past_end": [0, 200, T + 100], "short": [0, 200, T - 60], "negative_start": [-5, 200, T]}[tail]
+    computed = {"past_end": [(0, 200)], "short": [(0, 200), (200, T - 60)], "negative_start": [(200, T)]}[tail]
+    q, k, v = (t.to(DEV) for t in inputs.jagged_qkv(16, T + G, H, d, std=0.5 if kind == "hstu" else 1.0))
+    o = torch.full((T + G, H, d), SENTINEL, dtype=torch.bfloat16, device=DEV)
+    lse = torch.full((T + G, H), SENTINEL, dtype=torch.float32, device=DEV)
+    cu = torch.tensor(bounds, dtype=torch.int32, device=DEV)
+    L = eta.lib()
+    st = eta._stream_ptr()
+    max_len = 320
+    scale = eta.default_scale(d)
+    if kind == "varlen":
+        rc = L.attn_fwd_varlen(_vp(q), _vp(k), _vp(v), _vp(o), _vp(lse), _vp(cu), 2, max_len, T, H, d, scale, 1,
+                               eta.ETA_OUT_BF16, st)
+    else:
+        rc = L.hstu_fwd_jagged(_vp(q), _vp(k), _vp(v), _vp(o), _vp(cu), 2, max_len, T, H, d, 0.125, 1.0 / 256, st)
+    assert rc == 0
+    assert eta.status() == eta.ETA_DEV_BAD_CUSEQ
+    written = torch.zeros(T + G, dtype=torch.bool)
+    for a, b in computed:
+        written[a:b] = True
+        sub = lambda x: x[a:b].contiguous()
+        if kind == "varlen":
+            o_ref, lse_ref = oracle.attn_varlen(sub(q), sub(k), sub(v), [0, b - a], scale, True)
+            check_o(sub(o), o_ref, f"{kind} d={d} {tail} [{a},{b})")
+            check_lse(sub(lse), lse_ref, "lse")
+        else:
+            o_ref = oracle.hstu_jagged(sub(q), sub(k), sub(v), [0, b - a], 0.125, 1.0 / 256)
+            check_hstu(sub(o), o_ref, f"{kind} d={d} {tail} [{a},{b})")
+    untouched = ~written
+    assert torch.all(o.cpu()[untouched] == SENTINEL), "rows outside the computed sequences were written"
+    assert torch.all(lse.cpu()[untouched] == SENTINEL), "lse rows outside the computed sequences were written"
