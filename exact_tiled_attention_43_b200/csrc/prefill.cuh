@@ -155,9 +155,6 @@ struct PfCfg {
   static constexpr int QK_STEPS = ROW_BYTES / 32;        // K-steps of Q K^T: 32 bytes (16 bf16 or 32 e4m3) each
   static constexpr int PV_KEYS = 32 / ELT;               // keys per K-step of P V (8 TMEM columns of P)
   static constexpr int NST = (KV_TILE <= 16384) ? 8 : 4;  // K/V ring depth (each stage holds one tile)
-  // Of every 8 exp2 pairs, how many use the FMA-pipe polynomial instead of the MUFU.  Off: measured inside
-  // this kernel it costs more (issue slots, dependency chains) than the MUFU time it saves.
-  static constexpr int POLY_PAIRS = 0;
   // barriers: full/empty per stage; q_full[2], q_empty[2]; item_full[2], item_empty[2];
   // per tile {s_full, s_free, p_full, pv_done, o_free, mma_done}
   static constexpr int NBAR = 2 * NST + 4 + 4 + 2 * 6;
@@ -752,35 +749,24 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
         const uint64_t cs2 = f2pack(p.scale_log2, p.scale_log2), nm2 = f2pack(-msub, -msub);
         uint64_t rs_a = f2pack(0.f, 0.f), rs_b = f2pack(0.f, 0.f);
         float q0 = 0.f, q1 = 0.f;  // (F8) the previous pair, packed with the next one
-        // p = 2^(s * scale_log2 - m): pairs with (i % 8) < POLY_PAIRS go to the FMA-pipe polynomial on
-        // unmasked tiles, the rest (and every element of a masked tile) to the MUFU.
-        auto exp_row = [&](auto use_poly) {
+        // p = 2^(s * scale_log2 - m) on the MUFU; P packed to bf16 (or e4m3), the row sum kept in fp32
 #pragma unroll
-          for (int i = 0; i < BN / 2; ++i) {
-            const uint64_t x2 =
-                fma_x2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), cs2, nm2);
-            float x0, x1, p0, p1;
-            f2unpack(x2, x0, x1);
-            if (decltype(use_poly)::value && (i % 8) < C::POLY_PAIRS) {
-              exp2_poly_x2(x0, x1, p0, p1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
-            if (i & 1) rs_b = add_x2(rs_b, f2pack(p0, p1));
-            else rs_a = add_x2(rs_a, f2pack(p0, p1));
-            if constexpr (F8) {
-              // four keys per TMEM column: pairs 2m and 2m+1 go to column m
-              if (i & 1) pk[i >> 1] = pack_e4m3x4(q0, q1, p0, p1);
-              q0 = p0;
-              q1 = p1;
-            } else {
-              pk[i] = pack_bf16x2(p0, p1);
-            }
+        for (int i = 0; i < BN / 2; ++i) {
+          const uint64_t x2 = fma_x2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), cs2, nm2);
+          float x0, x1;
+          f2unpack(x2, x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          if (i & 1) rs_b = add_x2(rs_b, f2pack(p0, p1));
+          else rs_a = add_x2(rs_a, f2pack(p0, p1));
+          if constexpr (F8) {
+            // four keys per TMEM column: pairs 2m and 2m+1 go to column m
+            if (i & 1) pk[i >> 1] = pack_e4m3x4(q0, q1, p0, p1);
+            q0 = p0;
+            q1 = p1;
+          } else {
+            pk[i] = pack_bf16x2(p0, p1);
           }
-        };
-        if (need_mask) exp_row(std::false_type{});
-        else exp_row(std::true_type{});
+        }
         float r0a, r1a, r2a, r3a;
         f2unpack(rs_a, r0a, r1a);
         f2unpack(rs_b, r2a, r3a);

@@ -338,29 +338,4 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// 2^x for two values on the FMA pipe instead of the MUFU: Cody-Waite range reduction x = j + f with
-// j = round(x) (the 1.5 * 2^23 shifter), f in [-1/2, 1/2], 2^f by a cubic minimax polynomial (fitted by
-// csrc/fit_exp2_poly.py, max relative error 7.5e-5 over [-125, 8]), and 2^j added to the exponent field.
-// Inputs are clamped at -125 so the exponent never underflows; results below 2^-125 are not exact zeros.
-constexpr float EXP2_C0 = 0.9999281167984009f;
-constexpr float EXP2_C1 = 0.6932609677314758f;
-constexpr float EXP2_C2 = 0.24261054396629333f;
-constexpr float EXP2_C3 = 0.05517132207751274f;
-__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float &y0, float &y1) {
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  const uint64_t x = f2pack(x0, x1);
-  const uint64_t t = add_x2(x, f2pack(12582912.f, 12582912.f));      // round(x) in the low mantissa bits
-  const uint64_t r = add_x2(t, f2pack(-12582912.f, -12582912.f));    // round(x) as a float
-  const uint64_t f = fma_x2(r, f2pack(-1.f, -1.f), x);               // x - round(x)
-  uint64_t p = fma_x2(f2pack(EXP2_C3, EXP2_C3), f, f2pack(EXP2_C2, EXP2_C2));
-  p = fma_x2(p, f, f2pack(EXP2_C1, EXP2_C1));
-  p = fma_x2(p, f, f2pack(EXP2_C0, EXP2_C0));
-  float p0, p1, t0, t1;
-  f2unpack(p, p0, p1);
-  f2unpack(t, t0, t1);
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 }  // namespace eta
