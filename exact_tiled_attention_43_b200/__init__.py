@@ -14,7 +14,9 @@ Entry points (names follow the C ABI):
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
+import functools
 import math
 import os
 
@@ -151,10 +153,15 @@ def _check_buf(t, name, shape, dtypes, device):
 
 
 def _device_ctx(t):
-    """Makes t's GPU current for the call, so that the library and the default stream are t's."""
-    return _torch().cuda.device(t.device)
+    """Makes t's GPU current for the call, so that the library and the default stream are t's (nothing to
+    switch when it is current already, the usual case)."""
+    torch = _torch()
+    if t.device.index is None or t.device.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(t.device)
 
 
+@functools.lru_cache(maxsize=None)
 def default_scale(d: int) -> float:
     """The float32 value of 1/sqrt(d)."""
     import numpy as np

@@ -80,12 +80,49 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
+// The last few tensor maps this host thread encoded, keyed by everything that goes into one.  A call with
+// the same buffers and shapes as a recent one (the usual case in a loop) reuses the map instead of encoding
+// it again: the map holds only the address, sizes, strides, box and layout, so equal keys give equal maps.
+struct MapKey {
+  const void *base;
+  long long n1, n2;
+  int d, rows, elt, kind;  // kind: 0 dense, 1 packed, 2 page pool
+  bool operator==(const MapKey &o) const {
+    return base == o.base && n1 == o.n1 && n2 == o.n2 && d == o.d && rows == o.rows && elt == o.elt &&
+           kind == o.kind;
+  }
+};
+struct MapCache {
+  static constexpr int N = 16;
+  MapKey key[N];
+  CUtensorMap map[N];
+  bool used[N] = {};
+  int next = 0;
+  const CUtensorMap *find(const MapKey &k) const {
+    for (int i = 0; i < N; ++i)
+      if (used[i] && key[i] == k) return &map[i];
+    return nullptr;
+  }
+  void put(const MapKey &k, const CUtensorMap &m) {
+    key[next] = k;
+    map[next] = m;
+    used[next] = true;
+    next = (next + 1) % N;
+  }
+};
+thread_local MapCache t_maps;
+
 // bf16 rows of `d` elements; box = 64 elements (128 B, one swizzle span) x `rows` rows.
 // dense  : tensor [BH][N][d]      -> dims {d, N, BH},  box {64, rows, 1}
 // packed : tensor [T][H][d]       -> dims {d, H, T},   box {64, 1, rows}
 // `elt` bytes per element: 2 (bf16) or 1 (e4m3, mapped as bytes); the box always spans 128 bytes of a row.
 int encode_map(CUtensorMap *m, const void *base, bool packed, long long n1, long long n2, int d, int rows,
                int elt = 2) {
+  const MapKey key{base, n1, n2, d, rows, elt, packed ? 1 : 0};
+  if (const CUtensorMap *hit = t_maps.find(key)) {
+    *m = *hit;
+    return ETA_OK;
+  }
   EncodeTiledFn enc = get_encode();
   if (!enc) return ETA_ERR_CUDA;
   cuuint64_t dims[3], strides[2];
@@ -107,7 +144,27 @@ int encode_map(CUtensorMap *m, const void *base, bool packed, long long n1, long
   CUresult r = enc(m, (elt == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16), 3, const_cast<void *>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ETA_OK : ETA_ERR_CUDA;
+  if (r != CUDA_SUCCESS) return ETA_ERR_CUDA;
+  t_maps.put(key, *m);
+  return ETA_OK;
+}
+
+// Per-device, per-kernel launch set-up done once: the dynamic shared-memory limit and (for kernels that split
+// their registers between warpgroups) the check of the build's register count.  `state` is the calling
+// launcher's own table (one per kernel instance).
+template <typename Kern>
+int kernel_setup_once(std::atomic<int> (&state)[64], Kern kern, int smem, int want_regs) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ETA_ERR_CUDA;
+  if (state[dev].load(std::memory_order_acquire) == 1) return ETA_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ETA_ERR_CUDA;
+  if (want_regs > 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != want_regs) return ETA_ERR_CUDA;
+  }
+  state[dev].store(1, std::memory_order_release);  // a racing first call repeats the same set-up
+  return ETA_OK;
 }
 
 template <int MODE>
@@ -121,8 +178,8 @@ int launch_prefill_wide(const void *q, const void *k, const void *v, bool packed
   if ((rc = encode_map(&mv, v, packed, n1, n2, D, eta::WideCfg::BN)) != ETA_OK) return rc;
   auto kern = eta::prefill_wide_kernel<MODE>;
   constexpr int smem = eta::WideCfg::SMEM_BYTES;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return ETA_ERR_CUDA;
+  static std::atomic<int> ready[64];
+  if ((rc = kernel_setup_once(ready, kern, smem, 0)) != ETA_OK) return rc;
   kern<<<grid, eta::WideCfg::THREADS, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
 }
@@ -139,12 +196,10 @@ int launch_prefill(const void *q, const void *k, const void *v, bool packed, lon
   if ((rc = encode_map(&mv, v, packed, n1, n2, D, C::BN, C::ELT)) != ETA_OK) return rc;
   auto kern = eta::prefill_kernel<D, MODE, F8>;
   constexpr int smem = C::SMEM_BYTES;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return ETA_ERR_CUDA;
   // The kernel re-splits its registers between warpgroups (setmaxnreg); the split only adds up when the
   // build uses exactly PF_LAUNCH_REGS registers per thread, so refuse any other build.
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != eta::PF_LAUNCH_REGS) return ETA_ERR_CUDA;
+  static std::atomic<int> ready[64];
+  if ((rc = kernel_setup_once(ready, kern, smem, eta::PF_LAUNCH_REGS)) != ETA_OK) return rc;
   kern<<<grid, eta::PF_THREADS, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
 }
@@ -294,7 +349,9 @@ template <int D>
 int launch_decode(const eta::DecodeParams &p, cudaStream_t st) {
   constexpr int smem = 2 * eta::DEC_STAGES * eta::DEC_ROWS * D * 2;
   auto ks = eta::decode_split_kernel<D>;
-  if (cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return ETA_ERR_CUDA;
+  static std::atomic<int> ready[64];
+  int rc;
+  if ((rc = kernel_setup_once(ready, ks, smem, 0)) != ETA_OK) return rc;
   ks<<<dim3(p.max_splits, p.H, p.B), eta::DEC_THREADS, smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return ETA_ERR_CUDA;
   eta::decode_combine_kernel<D><<<dim3(p.H, p.B), D, 0, st>>>(p);
@@ -310,6 +367,11 @@ size_t decode_ws_bytes(int B, int H, int Lmax, int d) {
 // Page pool [num_pages, Hkv, page_size, d] bf16 viewed as a 3-D tensor {d, page_size, num_pages * Hkv}; box =
 // 64 elements (128 B, one swizzle span) x min(page_size, 32) rows x 1.
 int encode_paged_map(CUtensorMap *m, const void *base, int num_pages, int Hkv, int page_size, int d) {
+  const MapKey key{base, num_pages, Hkv, d, page_size, 2, 2};
+  if (const CUtensorMap *hit = t_maps.find(key)) {
+    *m = *hit;
+    return ETA_OK;
+  }
   EncodeTiledFn enc = get_encode();
   if (!enc) return ETA_ERR_CUDA;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)page_size, (cuuint64_t)num_pages * Hkv};
@@ -318,7 +380,9 @@ int encode_paged_map(CUtensorMap *m, const void *base, int num_pages, int Hkv, i
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ETA_OK : ETA_ERR_CUDA;
+  if (r != CUDA_SUCCESS) return ETA_ERR_CUDA;
+  t_maps.put(key, *m);
+  return ETA_OK;
 }
 
 template <int D>
@@ -330,7 +394,8 @@ int launch_decode_paged(const void *k_pages, const void *v_pages, const eta::Pag
   if ((rc = encode_paged_map(&mv, v_pages, p.num_pages, p.Hkv, p.page_size, D)) != ETA_OK) return rc;
   constexpr int smem = 1024 /*alignment slack*/ + 2 * eta::DPG_STAGES * eta::DPG_ROWS * D * 2;
   auto ks = eta::decode_paged_split_kernel<D>;
-  if (cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return ETA_ERR_CUDA;
+  static std::atomic<int> ready[64];
+  if ((rc = kernel_setup_once(ready, ks, smem, 0)) != ETA_OK) return rc;
   ks<<<dim3(p.max_splits, p.Hkv, p.B), eta::DPG_THREADS, smem, st>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return ETA_ERR_CUDA;
   eta::decode_combine_kernel<D><<<dim3(cp.H, cp.B), D, 0, st>>>(cp);
