@@ -155,6 +155,11 @@ struct PfCfg {
   static constexpr int QK_STEPS = ROW_BYTES / 32;        // K-steps of Q K^T: 32 bytes (16 bf16 or 32 e4m3) each
   static constexpr int PV_KEYS = 32 / ELT;               // keys per K-step of P V (8 TMEM columns of P)
   static constexpr int NST = (KV_TILE <= 16384) ? 8 : 4;  // K/V ring depth (each stage holds one tile)
+  // HSTU: of every 8 tanh pairs, how many go to the FMA-pipe polynomial (when in range) instead of the MUFU.
+  // At d = 64 both softmax warpgroups run at once and share the MUFU; moving 3 of 8 measured +10 % (jagged)
+  // and +13 % (dense) over 0, 2 or 4 of 8.  With P aliased into S (d >= 96) the warpgroups take turns and
+  // the MUFU is not the shared resource, so all stay on it.
+  static constexpr int TANH_FMA_PAIRS = ALIAS_P ? 0 : 3;
   // barriers: full/empty per stage; q_full[2], q_empty[2]; item_full[2], item_empty[2];
   // per tile {s_full, s_free, p_full, pv_done, o_free, mma_done}
   static constexpr int NBAR = 2 * NST + 4 + 4 + 2 * 6;
@@ -782,16 +787,39 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
             if (c > kmax) sr[c] = 0u;
         }
         const uint64_t ha2 = f2pack(p.hstu_half_alpha, p.hstu_half_alpha), ho2 = f2pack(p.hstu_out, p.hstu_out);
+        // tanh on the MUFU for every pair, or (TANH_FMA_PAIRS of every 8 pairs) on the FMA pipe by the degree-7
+        // polynomial, so that the two pipes share the work.  The polynomial holds for |alpha s / 2| <= 1: a
+        // warp takes the mixed loop only when every row's polynomial pairs are in that range.
+        bool mixed = false;
+        if constexpr (C::TANH_FMA_PAIRS > 0) {
+          float amax = 0.f;
 #pragma unroll
-        for (int i = 0; i < BN / 2; ++i) {
-          const uint64_t s2 = f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
-          float y0, y1;
-          f2unpack(mul_x2(s2, ha2), y0, y1);
-          const uint64_t h2 = mul_x2(s2, ho2);
-          float p0, p1;
-          f2unpack(fma_x2(h2, f2pack(tanh_approx(y0), tanh_approx(y1)), h2), p0, p1);
-          pk[i] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < BN / 2; ++i)
+            if ((i % 8) < C::TANH_FMA_PAIRS)
+              amax = max3f(amax, fabsf(__uint_as_float(sr[2 * i])), fabsf(__uint_as_float(sr[2 * i + 1])));
+          mixed = __all_sync(0xffffffffu, amax * fabsf(p.hstu_half_alpha) <= 1.f);
         }
+        auto pointwise = [&](auto with_poly) {
+#pragma unroll
+          for (int i = 0; i < BN / 2; ++i) {
+            const uint64_t s2 = f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+            const uint64_t y2 = mul_x2(s2, ha2);
+            const uint64_t h2 = mul_x2(s2, ho2);
+            uint64_t t2;
+            if (decltype(with_poly)::value && (i % 8) < C::TANH_FMA_PAIRS) {
+              t2 = tanh_poly_x2(y2);
+            } else {
+              float y0, y1;
+              f2unpack(y2, y0, y1);
+              t2 = f2pack(tanh_approx(y0), tanh_approx(y1));
+            }
+            float p0, p1;
+            f2unpack(fma_x2(h2, t2, h2), p0, p1);
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+        };
+        if (mixed) pointwise(std::true_type{});
+        else pointwise(std::false_type{});
       }
       if constexpr (!C::ALIAS_P) {
         // P_t's columns (and O_t) are free once the previous PV of this tile -- possibly the previous

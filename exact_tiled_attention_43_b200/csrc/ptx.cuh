@@ -338,4 +338,19 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
+// tanh(y) ~ y (c0 + c1 y^2 + c2 y^4 + c3 y^6) for |y| <= 1, on the FMA pipe for two values at once: the minimax
+// (absolute error) odd polynomial of degree 7 on [-1, 1], fitted by csrc/fit_tanh_poly.py (max error 3.3e-5 in
+// float32).  Callers keep |y| <= 1; outside that range the polynomial is not tanh.
+constexpr float TANH_C0 = 0.9996938109397888f;
+constexpr float TANH_C1 = -0.3288922607898712f;
+constexpr float TANH_C2 = 0.11541440337896347f;
+constexpr float TANH_C3 = -0.024654487147927284f;
+__device__ __forceinline__ uint64_t tanh_poly_x2(uint64_t y2) {
+  const uint64_t yy = mul_x2(y2, y2);
+  uint64_t p = fma_x2(f2pack(TANH_C3, TANH_C3), yy, f2pack(TANH_C2, TANH_C2));
+  p = fma_x2(p, yy, f2pack(TANH_C1, TANH_C1));
+  p = fma_x2(p, yy, f2pack(TANH_C0, TANH_C0));
+  return mul_x2(p, y2);
+}
+
 }  // namespace eta
