@@ -203,3 +203,24 @@ def test_split_tail_items(d, shape):
     o_ref, lse_ref = oracle.attn(q, k, v, scale, False)
     check_o(o, o_ref, f"split tail {shape} d={d}")
     check_lse(lse, lse_ref, "split tail lse")
+
+
+def test_same_buffers_different_shapes_back_to_back():
+    """The C ABI caches TMA tensor maps per host thread, keyed by buffer address and shape.  One storage viewed
+    as [1, 2, 512, 64] and then as [1, 4, 256, 64] (same base pointers, other sizes) must be mapped afresh each
+    time: both results equal the oracle, and repeating the first call after the second gives it again."""
+    base = [t.to(DEV) for t in inputs.dense_qkv(18, 1, 2, 512, 64)]
+    views_a = [t for t in base]
+    views_b = [t.view(1, 4, 256, 64) for t in base]
+    for causal in (False, True):
+        oa, la = eta.attn_fwd(*views_a, causal=causal)
+        ob, lb = eta.attn_fwd(*views_b, causal=causal)
+        oa2, la2 = eta.attn_fwd(*views_a, causal=causal)
+        assert eta.status() == 0
+        ra = oracle.attn(*views_a, eta.default_scale(64), causal)
+        rb = oracle.attn(*views_b, eta.default_scale(64), causal)
+        check_o(oa, ra[0], "shape A")
+        check_lse(la, ra[1], "shape A lse")
+        check_o(ob, rb[0], "shape B")
+        check_lse(lb, rb[1], "shape B lse")
+        assert torch.equal(oa, oa2) and torch.equal(la, la2)
