@@ -238,16 +238,14 @@ int plan_prefill(int mode, long long units, long long rows, int d, int causal, i
   // items all cost the same: when their count leaves a last wave at most half full, those last items are
   // split, so the last wave takes about half an item's time.  Launches too small to fill the GPU split every
   // item: causal ones (whose heaviest item sets the time of a single partial wave) with no more items than
-  // SMs, at every head dim up to 128 (B1 H8 N2048 d128: 196 -> 290 TFLOP/s); at d = 64 also non-causal
-  // ones with at most half as many items as SMs (at d = 128 a split item streams twice the K/V bytes per
-  // key step -- its tiles serve one warpgroup each).  Packed (varlen) launches follow the same rules on
-  // their item count.
+  // SMs, non-causal ones with at most half as many (B1 H8 N2048 d128: causal 196 -> 290 TFLOP/s,
+  // non-causal 357 -> 524).  Packed (varlen) launches follow the same rules on their item count.
   pl->whole = pl->items;
   if (mode != eta::MODE_HSTU && d <= 128 && rows > 128) {
     if (causal == 0 && pl->items > G) {
       const long long R = pl->items % G;
       if (R > 0 && 2 * R <= G) pl->whole = pl->items - R;
-    } else if ((causal != 0 && pl->items <= sms) || (d == 64 && causal == 0 && 2 * pl->items <= sms)) {
+    } else if ((causal != 0 && pl->items <= sms) || (causal == 0 && 2 * pl->items <= sms)) {
       pl->whole = 0;
     }
   }

@@ -15,12 +15,13 @@
 // Q tiles -- streaming the key/value tiles (128 rows each) its rows can see.  Causal tiles past the
 // diagonal are never loaded (the "after the diagonal: all zero, skip" class of the HSTU page's in-kernel
 // mask); only the diagonal tile and a ragged last tile evaluate a per-element mask.  The grid is persistent
-// (at most one CTA per SM): CTAs take items heaviest-first from a device counter and keep their pipeline
-// running across items, so the next item's Q, K/V and first QK^T overlap the current item's epilogue.
-// Non-causal dense launches whose item count leaves a last wave at most half full turn those last items
-// into split items: one 128-row Q tile whose key range is halved between the two softmax warpgroups, the
-// halves merged inside the CTA (exact: the same rescale identity as the online softmax), so the last wave
-// takes about half an item's time.
+// (at most one CTA per SM): CTAs take items from a device counter -- dense launches unit group by unit group
+// (so a group's K/V stay in L2), heaviest row block first inside a group -- and keep their pipeline running
+// across items, so the next item's Q, K/V and first QK^T overlap the current item's epilogue.  Split items
+// (one 128-row Q tile whose key range is halved between the two softmax warpgroups, the halves merged inside
+// the CTA: exact, the same rescale identity as the online softmax) serve two cases the host decides: the
+// last wave of a non-causal launch when at most half full, and every item of a launch too small to fill
+// the GPU.
 //
 // Roles (12 warps):
 //   warp 0      work fetcher + TMA producer: publishes each item to the other roles through a 2-deep ring,

@@ -240,8 +240,8 @@ ETA_API int attn_decode_noalloc(const void *q, const void *kcache, const void *v
  * NULL): *items = work items; *whole = items run whole, the other items - whole are each run as two split
  * halves (one Q tile, its key tiles divided between the CTA's two softmax warpgroups); *ctas = CTAs of the
  * persistent grid.  The split rule: non-causal launches whose last wave is at most half full split those
- * last items; causal launches with no more items than SMs, and at d = 64 non-causal ones with at most half
- * as many, split every item; HSTU and d = 256 never split.
+ * last items; causal launches with no more items than SMs, and non-causal ones with at most half as many,
+ * split every item; HSTU and d = 256 never split.
  * Returns 0, or ETA_ERR_HEAD_DIM / ETA_ERR_SHAPE / ETA_ERR_ARG as the planned call would.
  */
 ETA_API int eta_prefill_plan(int kind, long long units, long long rows, int d, int causal, int sms,

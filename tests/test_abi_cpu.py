@@ -135,12 +135,12 @@ def test_prefill_plan_split_policy():
     assert P("dense", 8, 2048, 64, False) == (64, 0, 128)
     assert P("dense", 32, 1024, 64, True) == (128, 0, 148)
     assert P("dense", 32, 1024, 64, False) == (128, 128, 128)  # 2 x 128 > 148: whole
-    # d = 96 and 128 split small causal launches too, but keep small non-causal ones whole; the non-causal
-    # last-wave rule still applies
+    # the same small-launch rule at d = 96 and 128; the non-causal last-wave rule still applies
     assert P("dense", 32, 1024, 128, True) == (128, 0, 148)
     assert P("dense", 8, 2048, 128, True) == (64, 0, 128)
     assert P("dense", 8, 2048, 96, True) == (64, 0, 128)
-    assert P("dense", 8, 2048, 128, False) == (64, 64, 64)
+    assert P("dense", 8, 2048, 128, False) == (64, 0, 128)
+    assert P("dense", 32, 1024, 128, False) == (128, 128, 128)  # 2 x 128 > 148: whole
     assert P("dense", 74, 1024, 128, True) == (296, 296, 148)  # more items than SMs: whole
     assert P("dense", 20, 2000, 128, False) == (160, 148, 148)  # 160 % 148 = 12 split
     assert P("dense", 148, 4096, 128, False) == (2368, 2368, 148)  # whole waves only

@@ -149,11 +149,11 @@ def test_more_items_than_sms(d, causal):
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("shape", [(1, 32, 1024), (1, 16, 1500), (1, 8, 2048), (3, 1, 700)])
 def test_split_all_items(d, causal, shape):
-    """Launches too small to fill the GPU: causal ones with no more items than SMs split every item (one Q
-    tile, its keys up to the diagonal halved between the warpgroups; a Q tile that sees one key tile stays
-    whole) at every head dim; at d = 64 non-causal ones with at most half as many items as SMs too, while
-    d = 96 and 128 run those unsplit.  (1,32,1024): 128 items; (1,16,1500): 96, ragged; (1,8,2048): 64;
-    (3,1,700): 9, ragged.  Every row compared, fp32 output."""
+    """Launches too small to fill the GPU split every item (one Q tile, its keys -- up to the diagonal when
+    causal -- halved between the warpgroups; a Q tile that sees one key tile stays whole): causal ones with
+    no more items than SMs, non-causal ones with at most half as many.  (1,32,1024): 128 items (non-causal:
+    whole); (1,16,1500): 96, ragged; (1,8,2048): 64; (3,1,700): 9, ragged.  Every row compared, fp32
+    output."""
     B, H, N = shape
     q, k, v = (t.to(DEV) for t in inputs.dense_qkv(14, B, H, N, d))
     scale = eta.default_scale(d)
