@@ -32,6 +32,10 @@
  *    valid for the call, a pipeline wait that ran out of time) never trap: the kernel
  *    keeps every access in bounds, records the first such condition in a device status word and carries
  *    on or returns.  Read it with eta_status().
+ *  - Per-device set-up is done once and kept for the process: each kernel's shared-memory limit and
+ *    register check on its first launch on a device, the allocation-free decode's scratch address, and (per
+ *    host thread) the TMA descriptors of recently used buffer shapes.  A device reset (cudaDeviceReset)
+ *    discards the first two; do not call the library on a device after resetting it.
  *  - Head dimension d: 64, 96 or 128 for every prefill call, 256 for softmax attention (attn_fwd,
  *    attn_fwd_varlen), 128 for the e4m3 call, 64 or 128 for decode.  The arithmetic is bf16 x bf16
  *    products accumulated in fp32 (tensor cores); softmax statistics and lse are fp32.
