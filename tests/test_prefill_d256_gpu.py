@@ -60,15 +60,16 @@ def test_d256_varlen_edge_lengths(causal):
     check_lse(lse, lse_ref, "d256 varlen lse")
 
 
-def test_d256_benchmark_config_sampled():
-    """B=4, H=16, N=4096, d=256 causal (the benchmark's d=256 line): sampled rows of four heads."""
+def test_d256_benchmark_config():
+    """B=4, H=16, N=4096, d=256 causal (the benchmark's d=256 line): every element and lse of every (batch,
+    head) compared with the oracle, one batch index at a time."""
     B, H, N = 4, 16, 4096
     q, k, v = inputs.dense_qkv(25, B, H, N, D, device=DEV)
     scale = eta.default_scale(D)
     o, lse = eta.attn_fwd(q, k, v, causal=True, scale=scale)
-    rows = sorted(set([0, 1, 63, 64, 127, 128, 129, 1000, 2047, 2048, 4094, 4095]))
-    for b, h in ((0, 0), (1, 7), (2, 15), (3, 3)):
-        sl = lambda x: x[b:b + 1, h:h + 1]
-        o_ref, lse_ref = oracle.attn(sl(q), sl(k), sl(v), scale, True, rows=rows)
-        check_o(sl(o)[:, :, rows], o_ref, f"d256 config b={b} h={h}")
-        check_lse(sl(lse)[:, :, rows], lse_ref, "d256 config lse")
+    assert eta.status() == 0
+    for b in range(B):
+        sl = lambda x: x[b:b + 1]
+        o_ref, lse_ref = oracle.attn(sl(q), sl(k), sl(v), scale, True)
+        check_o(sl(o), o_ref, f"d256 config b={b}")
+        check_lse(sl(lse), lse_ref, "d256 config lse")

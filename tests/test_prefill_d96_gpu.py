@@ -41,16 +41,16 @@ def test_d96_columns_past_the_head_dim_are_not_read():
     check_lse(lse[:, :1], lse_ref, "d96 next head NaN lse")
 
 
-def test_d96_benchmark_config_sampled():
-    """B=8, H=32, N=4096, d=96 causal (the benchmark's d=96 line): sampled rows of four (batch, head) pairs."""
+def test_d96_benchmark_config():
+    """B=8, H=32, N=4096, d=96 causal (the benchmark's d=96 line): every element and lse of every (batch,
+    head) compared with the oracle, one batch index at a time."""
     B, H, N = 8, 32, 4096
     q, k, v = inputs.dense_qkv(28, B, H, N, D, device=DEV)
     scale = eta.default_scale(D)
     o, lse = eta.attn_fwd(q, k, v, causal=True, scale=scale)
     assert eta.status() == 0
-    rows = sorted(set([0, 1, 127, 128, 255, 256, 257, 1000, 2047, 2048, 4094, 4095]))
-    for b, h in ((0, 0), (3, 17), (5, 31), (7, 5)):
-        sl = lambda x: x[b:b + 1, h:h + 1]
-        o_ref, lse_ref = oracle.attn(sl(q), sl(k), sl(v), scale, True, rows=rows)
-        check_o(sl(o)[:, :, rows], o_ref, f"d96 config b={b} h={h}")
-        check_lse(sl(lse)[:, :, rows], lse_ref, "d96 config lse")
+    for b in range(B):
+        sl = lambda x: x[b:b + 1]
+        o_ref, lse_ref = oracle.attn(sl(q), sl(k), sl(v), scale, True)
+        check_o(sl(o), o_ref, f"d96 config b={b}")
+        check_lse(sl(lse), lse_ref, "d96 config lse")

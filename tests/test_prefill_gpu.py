@@ -115,15 +115,28 @@ def test_grouped_schedule_ragged_last_group(causal):
     check_lse(lse, lse_ref, "grouped lse")
 
 
+def _sweep_rows(N, n=64):
+    """n query rows of an N-row sequence: the first and last rows, the rows on both sides of the first, the
+    middle and the last tile boundaries, and seeded random rows up to n."""
+    rows = {0, 1, 127, 128, 129, 255, 256, N // 2 - 1, N // 2, N - 129, N - 128, N - 2, N - 1}
+    rng = np.random.default_rng(N)
+    while len(rows) < n:
+        rows.add(int(rng.integers(0, N)))
+    return sorted(r for r in rows if 0 <= r < N)
+
+
 @pytest.mark.parametrize("N", [1024, 8192, 32768])
-def test_prefill_d128_sweep_sampled(N):
-    """N sweep at B=1, H=32, d=128, causal: sampled rows of three heads."""
+def test_prefill_d128_sweep(N):
+    """N sweep at B=1, H=32, d=128, causal, in the benchmark's launch configuration: 64 rows of every head
+    (rows are independent, so a row set checks the launch as a whole), every output element and lse of those
+    rows compared with the oracle."""
     q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, 1, 32, N, 128, device=DEV)
     scale = eta.default_scale(128)
     o, lse = eta.attn_fwd(q, k, v, causal=True, scale=scale)
     assert eta.status() == 0
-    rows = _sampled_rows(N)[:24]
-    for h in (0, 13, 31):
+    rows = _sweep_rows(N)
+    assert len(rows) == 64
+    for h in range(32):
         sl = lambda x: x[:, h:h + 1]
         o_ref, lse_ref = oracle.attn(sl(q), sl(k), sl(v), scale, True, rows=rows)
         check_o(sl(o)[:, :, rows], o_ref, f"sweep N={N} h={h}")
