@@ -367,7 +367,7 @@ def run_ours(args):
     # stream: the per-launch duration of the roofline is the mean of those.
     launch_ms = statistics.mean(per)
     achieved = step_flops / (launch_ms * 1e-3) / 1e12
-    traffic = recorded_traffic("prefill_d128_c3")
+    traffic = recorded_traffic("prefill_d128_b8")
 
     # ---- end to end through the public API with pinned host buffers.  Every step copies its own Q, K, V in
     # and its O and lse out.  Steps are pipelined the way a caller streaming batches would run them: the
@@ -658,8 +658,8 @@ def run_extras(args, eta, inputs, dev, flush, stream, ctx, peaks):
 
 CASES = {
     # name: (kind, shape) -- small named cases for profiler captures (no JSON line, just launches)
-    "prefill_d128_c3": ("dense_causal", dict(B=8, H=32, N=4096, d=128)),
-    "prefill_d64_headline": ("dense", dict(B=1, H=32, N=4096, d=64)),
+    "prefill_d128_b8": ("dense_causal", dict(B=8, H=32, N=4096, d=128)),
+    "prefill_d64_b1": ("dense", dict(B=1, H=32, N=4096, d=64)),
     "prefill_d64_b4": ("dense", dict(B=4, H=32, N=4096, d=64)),
     "prefill_d128_b2": ("dense", dict(B=2, H=32, N=4096, d=128)),
     "prefill_d96_b2": ("dense", dict(B=2, H=32, N=4096, d=96)),

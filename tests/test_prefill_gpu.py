@@ -77,8 +77,8 @@ def test_prefill_d64_full_config(causal):
     o, lse = eta.attn_fwd(q, k, v, causal=causal, scale=scale)
     assert eta.status() == 0
     o_ref, lse_ref = oracle.attn(q, k, v, scale, causal)
-    check_o(o, o_ref, f"C2 causal={causal}")
-    check_lse(lse, lse_ref, "C2 lse")
+    check_o(o, o_ref, f"B1 H32 N4096 d64 causal={causal}")
+    check_lse(lse, lse_ref, "B1 H32 N4096 d64 lse")
 
 
 def test_prefill_d128_full_config():
@@ -95,8 +95,8 @@ def test_prefill_d128_full_config():
     for b in range(B):
         sl = lambda x: x[b:b + 1]
         o_ref, lse_ref = oracle.attn(sl(q), sl(k), sl(v), scale, True)
-        check_o(sl(o), o_ref, f"C3 b={b}")
-        check_lse(sl(lse), lse_ref, f"C3 lse b={b}")
+        check_o(sl(o), o_ref, f"B8 H32 N4096 d128 b={b}")
+        check_lse(sl(lse), lse_ref, f"B8 H32 N4096 d128 lse b={b}")
 
 
 @pytest.mark.parametrize("causal", [False, True])

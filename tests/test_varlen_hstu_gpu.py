@@ -69,7 +69,7 @@ def test_hstu_full_config():
     o = eta.hstu_fwd_jagged(q, k, v, cu.to(DEV), 4096, 0.125, 1.0 / 4096)
     assert eta.status() == 0
     o_ref = oracle.hstu_jagged(q, k, v, cu, 0.125, 1.0 / 4096)
-    check_hstu(o, o_ref, "hstu C4")
+    check_hstu(o, o_ref, "hstu jagged 16 seqs H4 d64")
 
 
 @pytest.mark.parametrize("N", [4096, 8192])
