@@ -295,15 +295,18 @@ def run_reference(args):
     B, H, N, d = HEADLINE["B"], HEADLINE["H"], HEADLINE["N"], HEADLINE["d"]
     q, k, v = inputs.dense_qkv(inputs.PREFILL_D128, B, H, N, d)
     scale = float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))
-    # each step: one (batch, head) unit, causal, every 32nd query row (a bounded CPU time per step); the
-    # units rotate through the batch so that successive steps read different data
-    rows = list(range(0, N, 32))
-    step_flops = sum(4.0 * (r + 1) * d for r in rows)
-    units = [(b, h) for b in range(B) for h in range(0, H, 7)]
+    # each step: four (batch, head) units of one batch index, causal, every 8th query row (a bounded CPU time
+    # per step, ~0.1 s, large enough for the oracle's threads to share); the batch index rotates so that
+    # successive steps read different data
+    rows = list(range(0, N, 8))
+    per_unit = sum(4.0 * (r + 1) * d for r in rows)
+    step_units = 4
+    step_flops = per_unit * step_units
 
     def step(i):
-        b, h = units[i % len(units)]
-        oracle.attn(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1], scale, True, rows=rows)
+        b = i % B
+        hs = slice((i * step_units) % H, (i * step_units) % H + step_units)
+        oracle.attn(q[b:b + 1, hs], k[b:b + 1, hs], v[b:b + 1, hs], scale, True, rows=rows)
 
     for i in range(args.warmup):
         step(i)
@@ -313,8 +316,8 @@ def run_reference(args):
     el = time.perf_counter() - t0
     val = step_flops * args.steps / el / 1e12
     cores = oracle.num_threads()
-    sample = (f"per step: 1 of {B * H} (batch, head) units, every 32nd query row ({len(rows)} rows), causal, "
-              f"N={N}, d={d}")
+    sample = (f"per step: {step_units} of {B * H} (batch, head) units, every 8th query row ({len(rows)} rows "
+              f"each), causal, N={N}, d={d}")
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
