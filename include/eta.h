@@ -16,12 +16,19 @@
  *   attn_decode                  one new query per (batch, head) against a long KV cache.
  *       "AI attention complexity ledger", section "带宽账：decode 阶段的真正瓶颈"
  *       (s_j = q . k_j over all cached keys, o = sum_j p_j v_j; HBM-bound).
+ *   attn_fwd_fp8                 attn_fwd on e4m3 inputs with per-tensor descales ("FlashAttention (TH)",
+ *       section "FlashAttention-3").
+ *   attn_decode_paged            the decode step with grouped query heads over a paged KV cache.
+ *   attn_decode_noalloc          attn_decode with its scratch in the library's own device array.
+ *   eta_prefill_plan, eta_prefill_sched_group, eta_status, eta_strerror, eta_set_wait_timeout_ns,
+ *   eta_selftest_wait_timeout    host-side queries, the device status word and the bounded-wait limit.
  *
  * Conventions shared by every call
  * --------------------------------
  *  - Pointers named q, k, v, o, kcache, vcache, lse, cu_seqlens, kv_lens, workspace are DEVICE pointers
  *    (cudaMalloc'd or equivalent) on the current CUDA device.  The caller owns every buffer; the library
- *    allocates no device memory and keeps no per-call state.
+ *    allocates no device memory when called: its only device memory is the module's own static data (the
+ *    status word, the prefill work counters and the allocation-free decode's scratch array).
  *  - bf16 means IEEE bfloat16 stored as 16-bit words; all tensors are contiguous, row-major, with the
  *    layouts given per call.  q, k, v, o and the caches must be 16-byte aligned.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only enqueues work on it and
