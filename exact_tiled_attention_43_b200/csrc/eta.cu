@@ -175,7 +175,7 @@ int launch_prefill_wide(const void *q, const void *k, const void *v, bool packed
   int rc;
   if ((rc = encode_map(&mq, q, packed, n1, n2, D, eta::PF_BM)) != ETA_OK) return rc;
   if ((rc = encode_map(&mk, k, packed, n1, n2, D, eta::WideCfg::BN)) != ETA_OK) return rc;
-  if ((rc = encode_map(&mv, v, packed, n1, n2, D, eta::WideCfg::BN)) != ETA_OK) return rc;
+  if ((rc = encode_map(&mv, v, packed, n1, n2, D, eta::WideCfg::V_ROWS)) != ETA_OK) return rc;
   auto kern = eta::prefill_wide_kernel<MODE>;
   constexpr int smem = eta::WideCfg::SMEM_BYTES;
   static std::atomic<int> ready[64];

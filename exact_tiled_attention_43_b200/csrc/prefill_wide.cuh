@@ -7,9 +7,13 @@
 //
 // Why a kernel of its own: a 128-row O accumulator of 256 fp32 columns takes half of TMEM, so a CTA holds one
 // Q tile, not two.  Layout per CTA:
-//   TMEM   S_0 [0,64), S_1 [64,128) (double-buffered 128 x 64 scores; P of a key tile is written over the
-//          first 32 columns of its S buffer), O [256,512).
-//   SMEM   Q (128 x 256 bf16, 64 KB) + a 4-stage ring of 64-key K and V tiles (32 KB each).
+//   TMEM   S_0 [0,128), S_1 [128,256) (double-buffered 128 x 128 scores; P of a key tile is written over the
+//          first 64 columns of its S buffer), O [256,512).
+//   SMEM   Q (128 x 256 bf16, 64 KB) + a ring of five 32 KB slots.  A key tile (128 keys) is K in two slots
+//          (two 64-column chunks each) and V in two slots (64 keys with all four column chunks each), so a
+//          QK^T is 16 MMAs of N = 128 and a PV 8 of N = 256, and each slot is handed back to the producer as
+//          soon as the MMAs that read it are complete: the loads of the next tile start while the current
+//          one is still being multiplied.
 //   warps  0: work fetcher + TMA producer; 1: MMA issuer (one thread); 2-3: no role; 4-7: softmax (thread r
 //          owns query row r = TMEM lane r).
 // The issuer runs PV(j) then QK^T(j+2) into the buffer PV(j) has just read, with no wait between them
@@ -24,31 +28,41 @@ namespace eta {
 
 struct WideCfg {
   static constexpr int D = 256;
-  static constexpr int BN = 64;                          // keys per K/V tile
+  static constexpr int BN = 128;                         // keys per key tile
   static constexpr int KCH = D / 64;                     // 128-byte column chunks per row
   static constexpr int Q_CHUNK = PF_BM * 128;            // 128 rows x 128 B
   static constexpr int Q_TILE = KCH * Q_CHUNK;           // 64 KB
-  static constexpr int KV_CHUNK = BN * 128;              // 64 rows x 128 B
-  static constexpr int KV_TILE = KCH * KV_CHUNK;         // 32 KB
-  static constexpr int NST = 4;                          // K/V ring depth
+  static constexpr int K_CHUNK = BN * 128;               // one column chunk of a K tile: 128 keys x 128 B
+  // The K/V ring is made of equal slots.  A K slot holds KC_PER_SLOT column chunks of one key tile (all 128
+  // keys); a V slot holds V_ROWS keys of one key tile with every column chunk (V_CHUNK bytes each), so the
+  // QK^T k-steps and the PV k-steps each consume their slots in order and release them one by one.  (16 KB
+  // slots -- ten of them -- measured 16 % slower: twice the barrier waits and commits on the issuer thread.)
+  static constexpr int KC_PER_SLOT = 2;
+  static constexpr int SLOT = KC_PER_SLOT * K_CHUNK;
+  static constexpr int V_ROWS = SLOT / (KCH * 128);      // 64 keys
+  static constexpr int V_CHUNK = V_ROWS * 128;
+  static constexpr int K_SLOTS = KCH / KC_PER_SLOT;      // slots per K tile
+  static constexpr int V_SLOTS = BN / V_ROWS;            // slots per V tile
+  static constexpr int NSLOT = 5;                        // 160 KB of ring
   static constexpr int NSB = 2;                          // S buffers
   static constexpr uint32_t TM_O = 256;
   static constexpr int THREADS = 256;
-  // barriers: full/empty per stage; q_full, q_empty; item_full[2], item_empty[2]; s_full, p_full and pv_done
+  // barriers: full/empty per slot; q_full, q_empty; item_full[2], item_empty[2]; s_full, p_full and pv_done
   // per S buffer; o_free; mma_done.  The S, P and PV barriers are per buffer because with two S buffers the
   // softmax runs up to a key tile ahead of the tensor core: one shared barrier could then be two phases from
   // its waiter, and a parity wait cannot tell that from being done.  Per buffer, the previous phase of each
   // barrier is always complete when it is waited on (a key tile's QK^T is issued after the PV two tiles back).
-  static constexpr int NBAR = 2 * NST + 2 + 4 + 3 * NSB + 2;
-  static constexpr int SMEM_BYTES = 1024 + Q_TILE + NST * KV_TILE + NBAR * 8 + 2 * (int)sizeof(PfItem) + 16;
+  static constexpr int NBAR = 2 * NSLOT + 2 + 4 + 3 * NSB + 2;
+  static constexpr int SMEM_BYTES = 1024 + Q_TILE + NSLOT * SLOT + NBAR * 8 + 2 * (int)sizeof(PfItem) + 16;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+  static_assert(K_SLOTS * KC_PER_SLOT == KCH && V_SLOTS * V_ROWS == BN && V_ROWS % 16 == 0, "slot shapes");
 };
 
 struct WideSmem {
   using C = WideCfg;
   static constexpr int OFF_KV = C::Q_TILE;
-  static constexpr int OFF_BAR = OFF_KV + C::NST * C::KV_TILE;
-  static constexpr int B_FULL = 0, B_EMPTY = C::NST, B_QFULL = 2 * C::NST, B_QEMPTY = B_QFULL + 1,
+  static constexpr int OFF_BAR = OFF_KV + C::NSLOT * C::SLOT;
+  static constexpr int B_FULL = 0, B_EMPTY = C::NSLOT, B_QFULL = 2 * C::NSLOT, B_QEMPTY = B_QFULL + 1,
                        B_ITEM_FULL = B_QEMPTY + 1, B_ITEM_EMPTY = B_ITEM_FULL + 2, B_S_FULL = B_ITEM_EMPTY + 2,
                        B_P_FULL = B_S_FULL + C::NSB, B_PV_DONE = B_P_FULL + C::NSB, B_O_FREE = B_PV_DONE + C::NSB,
                        B_MMA_DONE = B_O_FREE + 1, B_END = B_MMA_DONE + 1;
@@ -165,29 +179,56 @@ __device__ __forceinline__ void wide_control(const CUtensorMap &tmQ, const CUten
             tma_load_3d(dst, &tmQ, sm.q_full(), 64 * c, it.r0, it.bh);
         }
         ++q_issued;
-        for (int i = 0; ok && i < 2 * it.n0; ++i) {
-          const int st = kv_issued % C::NST;
-          ok = mbar_wait(sm.empty(st), ((kv_issued / C::NST) & 1) ^ 1, sm.abort_flag(), p.wait_ns);
-          if (!ok) break;
-          const int jt = i >> 1;
-          const CUtensorMap *m = (i & 1) ? &tmV : &tmK;
-          mbar_arrive_expect_tx(sm.full(st), C::KV_TILE);
+        // Slots in the order the issuer consumes them: K_0, K_1, then V_j, K_{j+2} for each key tile j.
+        auto acquire = [&]() {
+          const int st = kv_issued % C::NSLOT;
+          if (!mbar_wait(sm.empty(st), ((kv_issued / C::NSLOT) & 1) ^ 1, sm.abort_flag(), p.wait_ns)) return -1;
+          mbar_arrive_expect_tx(sm.full(st), C::SLOT);
+          return st;
+        };
+        auto load_k = [&](int j) {
+          for (int s = 0; s < C::K_SLOTS; ++s) {
+            const int st = acquire();
+            if (st < 0) return false;
 #pragma unroll
-          for (int c = 0; c < C::KCH; ++c) {
-            uint8_t *dst = sm.sKV() + st * C::KV_TILE + c * C::KV_CHUNK;
-            if constexpr (PACKED)
-              tma_load_3d(dst, m, sm.full(st), 64 * c, it.h, it.seq_start + jt * C::BN);
-            else
-              tma_load_3d(dst, m, sm.full(st), 64 * c, jt * C::BN, it.bh);
+            for (int c2 = 0; c2 < C::KC_PER_SLOT; ++c2) {
+              uint8_t *dst = sm.sKV() + st * C::SLOT + c2 * C::K_CHUNK;
+              const int x = 64 * (s * C::KC_PER_SLOT + c2);
+              if constexpr (PACKED)
+                tma_load_3d(dst, &tmK, sm.full(st), x, it.h, it.seq_start + j * C::BN);
+              else
+                tma_load_3d(dst, &tmK, sm.full(st), x, j * C::BN, it.bh);
+            }
+            ++kv_issued;
           }
-          ++kv_issued;
-        }
+          return true;
+        };
+        auto load_v = [&](int j) {
+          for (int s = 0; s < C::V_SLOTS; ++s) {
+            const int st = acquire();
+            if (st < 0) return false;
+            const int r = j * C::BN + s * C::V_ROWS;
+#pragma unroll
+            for (int c = 0; c < C::KCH; ++c) {
+              uint8_t *dst = sm.sKV() + st * C::SLOT + c * C::V_CHUNK;
+              if constexpr (PACKED)
+                tma_load_3d(dst, &tmV, sm.full(st), 64 * c, it.h, it.seq_start + r);
+              else
+                tma_load_3d(dst, &tmV, sm.full(st), 64 * c, r, it.bh);
+            }
+            ++kv_issued;
+          }
+          return true;
+        };
+        const int n = it.n0;
+        ok = load_k(0) && (n < 2 || load_k(1));
+        for (int j = 0; ok && j < n; ++j) ok = load_v(j) && (j + 2 >= n || load_k(j + 2));
       }
       if (!retired) retire();
       if (!ok) {
         if (q_issued > 0) mbar_wait(sm.q_full(), (q_issued - 1) & 1, nullptr, p.wait_ns);
-        for (int i = max(0, kv_issued - C::NST); i < kv_issued; ++i)
-          mbar_wait(sm.full(i % C::NST), (i / C::NST) & 1, nullptr, p.wait_ns);
+        for (int i = max(0, kv_issued - C::NSLOT); i < kv_issued; ++i)
+          mbar_wait(sm.full(i % C::NSLOT), (i / C::NSLOT) & 1, nullptr, p.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -197,31 +238,60 @@ __device__ __forceinline__ void wide_control(const CUtensorMap &tmQ, const CUten
       constexpr uint32_t ID_PV = idesc_bf16_f32(PF_BM, C::D, true);
       const uint32_t sQa = smem_u32(sm.sQ()), sKVa = smem_u32(sm.sKV());
       const uint64_t dQ = sdesc_sw128(sQa, 16, 1024), dK = sdesc_sw128(sKVa, 16, 1024);
-      const uint64_t dV = sdesc_sw128(sKVa, C::KV_CHUNK, 1024);
-      // S_b = Q K^T : 16 k-steps of 16 head-dim elements (32 bytes inside a 128-byte swizzled row)
-      auto issue_s = [&](int b, int st) {
-        const uint64_t db = dK + (uint64_t)((st * C::KV_TILE) >> 4);
-        const uint32_t dt = tmem + (uint32_t)(C::BN * b);
-        eta_static_for<C::D / 16>([&](auto kk_c) {
-          constexpr int kk = decltype(kk_c)::value;
-          constexpr uint32_t a_off = ((uint32_t)(kk >> 2) * C::Q_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
-          constexpr uint32_t b_off = ((uint32_t)(kk >> 2) * C::KV_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
-          mma_ss_off<a_off, b_off>(dt, dQ, db, ID_QK, kk > 0 ? 1u : 0u);
-        });
+      const uint64_t dV = sdesc_sw128(sKVa, C::V_CHUNK, 1024);
+      int g = 0;  // ring slots consumed, over all items
+      bool ok = true;
+      auto slot_wait = [&]() {
+        ok = ok && mbar_wait(sm.full(g % C::NSLOT), (g / C::NSLOT) & 1, sm.abort_flag(), p.wait_ns);
+        if (ok) tc_fence_after();
+        return (uint64_t)(((g % C::NSLOT) * C::SLOT) >> 4);
       };
-      // O += P_b V : 4 k-steps of 16 keys (8 TMEM columns of packed bf16 P, 16 rows = 2048 B of V), N = 256
-      auto issue_pv = [&](int b, int st, bool acc) {
-        const uint64_t db = dV + (uint64_t)((st * C::KV_TILE) >> 4);
+      auto slot_release = [&]() {
+        mma_commit(sm.empty(g % C::NSLOT));
+        ++g;
+      };
+      // S_b = Q K^T : 16 k-steps of 16 head-dim elements (32 bytes inside a 128-byte swizzled row), N = 128;
+      // each K slot is released once the k-steps that read it are complete.
+      auto issue_s = [&](int b) {
+        const uint32_t dt = tmem + (uint32_t)(C::BN * b);
+        eta_static_for<C::K_SLOTS>([&](auto s_c) {
+          constexpr int s = decltype(s_c)::value;
+          const uint64_t so = slot_wait();
+          if (!ok) return;
+          const uint64_t db = dK + so;
+          eta_static_for<4 * C::KC_PER_SLOT>([&](auto i_c) {
+            constexpr int kk = s * 4 * C::KC_PER_SLOT + decltype(i_c)::value;
+            constexpr uint32_t a_off = ((uint32_t)(kk >> 2) * C::Q_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
+            constexpr uint32_t b_off =
+                ((uint32_t)((kk >> 2) % C::KC_PER_SLOT) * C::K_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
+            mma_ss_off<a_off, b_off>(dt, dQ, db, ID_QK, kk > 0 ? 1u : 0u);
+          });
+          slot_release();
+        });
+        if (ok) mma_commit(sm.s_full(b));
+        return ok;
+      };
+      // O += P_b V : 8 k-steps of 16 keys (8 TMEM columns of packed bf16 P; 16 rows = 2048 B of each column
+      // chunk of a V slot), N = 256
+      auto issue_pv = [&](int b, bool acc) {
         const uint32_t tP = tmem + (uint32_t)(C::BN * b);
         const uint32_t acc0 = acc ? 1u : 0u;
-        eta_static_for<C::BN / 16>([&](auto kk_c) {
-          constexpr int kk = decltype(kk_c)::value;
-          constexpr uint32_t ta_off = 8u * kk, b_off = (2048u * kk) / 16u;
-          mma_ts_off<ta_off, b_off>(tmem + C::TM_O, tP, db, ID_PV, kk > 0 ? 1u : acc0);
+        eta_static_for<C::V_SLOTS>([&](auto s_c) {
+          constexpr int s = decltype(s_c)::value;
+          const uint64_t so = slot_wait();
+          if (!ok) return;
+          const uint64_t db = dV + so;
+          eta_static_for<C::V_ROWS / 16>([&](auto i_c) {
+            constexpr int ki = decltype(i_c)::value;
+            constexpr int kk = s * (C::V_ROWS / 16) + ki;
+            constexpr uint32_t ta_off = 8u * kk, b_off = (2048u * ki) / 16u;
+            mma_ts_off<ta_off, b_off>(tmem + C::TM_O, tP, db, ID_PV, kk > 0 ? 1u : acc0);
+          });
+          slot_release();
         });
+        return ok;
       };
-      int gs = 0, gp = 0, go = 0, kv_base = 0;  // S issued, PV issued, items done (over all items)
-      bool ok = true;
+      int gs = 0, gp = 0, go = 0;  // S issued, PV issued, items done (over all items)
       for (int k = 0; ok; ++k) {
         ok = mbar_wait(sm.item_full(k & 1), (k >> 1) & 1, sm.abort_flag(), p.wait_ns);
         if (!ok) break;
@@ -231,38 +301,27 @@ __device__ __forceinline__ void wide_control(const CUtensorMap &tmQ, const CUten
         const int n = it.n0;  // >= 1
         ok = mbar_wait(sm.q_full(), k & 1, sm.abort_flag(), p.wait_ns);
         if (!ok) break;
-        auto kv_wait = [&](int i) {
-          const int g = kv_base + i;
-          return mbar_wait(sm.full(g % C::NST), (g / C::NST) & 1, sm.abort_flag(), p.wait_ns);
-        };
-        auto kv_stage = [&](int i) { return (kv_base + i) % C::NST; };
+        tc_fence_after();
         // S(j) goes to buffer (gs of that S) % NSB.  The first two of an item follow the previous item's last
         // PVs in issue order, which is all the buffers need.
         auto s_step = [&](int j) {
-          if (!kv_wait(2 * j)) return false;
-          tc_fence_after();
-          issue_s(gs % C::NSB, kv_stage(2 * j));
-          mma_commit(sm.s_full(gs % C::NSB));
-          mma_commit(sm.empty(kv_stage(2 * j)));
+          if (!issue_s(gs % C::NSB)) return false;
           ++gs;
           if (j == n - 1) mma_commit(sm.q_empty());  // every QK^T of this item is issued
           return true;
         };
         ok = s_step(0) && (n < 2 || s_step(1));
         for (int j = 0; ok && j < n; ++j) {
-          ok = kv_wait(2 * j + 1) &&
-               mbar_wait(sm.p_full(gp % C::NSB), (gp / C::NSB) & 1, sm.abort_flag(), p.wait_ns) &&
+          ok = mbar_wait(sm.p_full(gp % C::NSB), (gp / C::NSB) & 1, sm.abort_flag(), p.wait_ns) &&
                (j > 0 || go == 0 || mbar_wait(sm.o_free(), (go - 1) & 1, sm.abort_flag(), p.wait_ns));
           if (!ok) break;
           tc_fence_after();
-          issue_pv(gp % C::NSB, kv_stage(2 * j + 1), j > 0);
+          if (!issue_pv(gp % C::NSB, j > 0)) break;
           mma_commit(sm.pv_done(gp % C::NSB));
-          mma_commit(sm.empty(kv_stage(2 * j + 1)));
           ++gp;
           if (j + 2 < n) ok = s_step(j + 2);  // into the buffer PV(j) has just read, in issue order after it
         }
         ++go;
-        kv_base += 2 * n;
       }
       mma_commit(sm.mma_done());
       mbar_wait(sm.mma_done(), 0, nullptr, p.wait_ns);
@@ -441,7 +500,7 @@ __global__ void __launch_bounds__(WideCfg::THREADS, 1)
   WideSmem sm(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NST; ++i) {
+    for (int i = 0; i < C::NSLOT; ++i) {
       mbar_init(sm.full(i), 1);
       mbar_init(sm.empty(i), 1);
     }
