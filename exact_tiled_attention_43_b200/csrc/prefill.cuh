@@ -36,8 +36,10 @@
 //   D = 64: P_t has its own columns [384+64t, 448+64t); issuer 1+t serves Q tile t and issues the next
 //           S_t as soon as the softmax has copied S_t to registers.  Two Q slots in shared memory: the
 //           next item's Q tiles load while the current item runs.
-//   D = 96, 128 (and e4m3 at 128): TMEM is full; P_t overwrites the first columns of S_t and one issuer
-//           (warp 1) runs
+//   D = 96: 96-key tiles, so S_t uses 96 of its 128 columns and O_t 96 of its 128; P_t (48 columns) lives
+//           in those spare columns (keys [0, 64) after S_t, keys [64, 96) after O_t) and the D = 64 flow
+//           applies: one issuer per tile, the next S_t issued as soon as S_t has been read.
+//   D = 128 (and e4m3): TMEM is full; P_t overwrites the first columns of S_t and one issuer (warp 1) runs
 //           PV_0(j), S_0(j+1), PV_1(j), S_1(j+1) with no wait between a PV and the next QK^T: tcgen05.mma
 //           operations issued by one thread execute in issue order, so the QK^T's writes follow the PV's
 //           reads of P, and the QK^T's commit also covers the PV (a softmax that has seen the new S may
@@ -138,7 +140,8 @@ struct PfCfg {
   // Keys per K/V tile.  (At d = 128, 64-key tiles would leave TMEM room for a separate P -- 2 S + 2 O + 2 P =
   // 128 + 256 + 64 columns -- so that the next QK^T need not follow the PV that reads P; measured, the
   // halved tiles cost more in per-tile overhead and MMA latency than that saves: 11 % slower.)
-  static constexpr int BN = 128;
+  // (d = 96: 96-key tiles, so that a separate P fits in TMEM; see P_IN_HOLES.)
+  static constexpr int BN = (D == 96 && !F8) ? 96 : 128;
   static constexpr int P_COLS = BN * ELT / 4;            // TMEM columns of one tile's P (bf16 or e4m3, packed)
   // 128-byte column chunks per row.  A row that is not a whole number of chunks (d = 96: 192 bytes) has its
   // last chunk half filled by the TMA's zero fill past the tensor's inner extent; the MMAs never read the
@@ -146,8 +149,13 @@ struct PfCfg {
   static constexpr int KCH = (ROW_BYTES + 127) / 128;
   // TMEM columns reserved per O tile: the head dim rounded up to whole chunks (d = 96 keeps 128).
   static constexpr int O_COLS = KCH * 128 / ELT;
-  // P overwrites S's first columns only when S, O and P of both tiles do not fit in 512 TMEM columns.
-  static constexpr bool ALIAS_P = (2 * BN + 2 * O_COLS + 2 * P_COLS) > 512;
+  // S_t takes 128 columns from S_STRIDE * t (BN of them used).  d = 96: P_t goes into the spare columns, keys
+  // [0, 64) into S_t's [96, 128) and keys [64, 96) into O_t's [96, 112), so that every tile has its own P
+  // (no PV -> next QK^T chain) while S and O keep 128-column slots.  Otherwise P overwrites S's first columns
+  // when S, O and P of both tiles do not fit in 512 TMEM columns.
+  static constexpr int S_STRIDE = 128;
+  static constexpr bool P_IN_HOLES = (D == 96 && !F8);
+  static constexpr bool ALIAS_P = !P_IN_HOLES && (2 * BN + 2 * O_COLS + 2 * P_COLS) > 512;
   static constexpr int N_ISSUERS = ALIAS_P ? 1 : 2;
   static constexpr int Q_CHUNK = PF_BM * 128;            // 128 rows x 128 B
   static constexpr int Q_TILE = KCH * Q_CHUNK;           // one 128 x D Q tile
@@ -155,11 +163,13 @@ struct PfCfg {
   static constexpr int KV_TILE = KCH * KV_CHUNK;         // one BN x D K or V tile
   static constexpr int QK_STEPS = ROW_BYTES / 32;        // K-steps of Q K^T: 32 bytes (16 bf16 or 32 e4m3) each
   static constexpr int PV_KEYS = 32 / ELT;               // keys per K-step of P V (8 TMEM columns of P)
-  static constexpr int NST = (KV_TILE <= 16384) ? 8 : 4;  // K/V ring depth (each stage holds one tile)
+  // K/V ring depth (each stage holds one tile).  d = 96 takes six 24 KB stages and one Q slot (four stages
+  // and two Q slots measured 6 % slower at B8 H32 N4096 causal, 8 % non-causal).
+  static constexpr int NST = (KV_TILE <= 16384) ? 8 : (P_IN_HOLES ? 6 : 4);
   // HSTU: of every 8 tanh pairs, how many go to the FMA-pipe polynomial (when in range) instead of the MUFU.
-  // At d = 64 both softmax warpgroups run at once and share the MUFU; moving 3 of 8 measured +10 % (jagged)
-  // and +13 % (dense) over 0, 2 or 4 of 8.  With P aliased into S (d >= 96) the warpgroups take turns and
-  // the MUFU is not the shared resource, so all stay on it.
+  // With a separate P (d = 64, 96) both softmax warpgroups run at once and share the MUFU; moving 3 of 8
+  // measured +10 % (jagged) and +13 % (dense) over 0, 2 or 4 of 8 at d = 64.  With P aliased into S (d = 128)
+  // the warpgroups take turns and the MUFU is not the shared resource, so all stay on it.
   static constexpr int TANH_FMA_PAIRS = ALIAS_P ? 0 : 3;
   // barriers: full/empty per stage; q_full[2], q_empty[2]; item_full[2], item_empty[2];
   // per tile {s_full, s_free, p_full, pv_done, o_free, mma_done}
@@ -170,10 +180,12 @@ struct PfCfg {
   // loaded while the current item still runs and its first QK^T is ready when the softmax gets to it.
   static constexpr int QSLOTS = (SMEM_FIXED + 4 * Q_TILE <= 227 * 1024) ? 2 : 1;
   static constexpr int SMEM_BYTES = SMEM_FIXED + QSLOTS * 2 * Q_TILE;
-  // TMEM columns: S_t at BN*t, O_t at TM_O + O_COLS*t, P_t at TM_P + P_COLS*t (or S_t's first columns if ALIAS_P)
-  static constexpr uint32_t TM_O = 2 * BN;
-  static constexpr uint32_t TM_P = 2 * BN + 2 * O_COLS;
-  static_assert(TM_P + (ALIAS_P ? 0 : 2 * P_COLS) <= 512, "TMEM columns");
+  // TMEM columns: S_t at S_STRIDE*t, O_t at TM_O + O_COLS*t, P_t at TM_P + P_COLS*t (S_t's first columns if
+  // ALIAS_P; S_t's and O_t's spare columns if P_IN_HOLES)
+  static constexpr uint32_t TM_O = 2 * S_STRIDE;
+  static constexpr uint32_t TM_P = 2 * S_STRIDE + 2 * O_COLS;
+  static_assert(BN <= S_STRIDE && TM_P + ((ALIAS_P || P_IN_HOLES) ? 0 : 2 * P_COLS) <= 512, "TMEM columns");
+  static_assert(!P_IN_HOLES || (BN == 96 && O_COLS == 128 && P_COLS == 48), "d = 96 P layout");
   static_assert(ROW_BYTES % 32 == 0 && D % 32 == 0 && D <= O_COLS, "head dim: whole K-steps and TMEM loads");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 };
@@ -416,7 +428,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
       auto issue_s = [&](int t, int st) {
         const uint64_t da = dQ + (uint64_t)((q_off + (uint32_t)(t * C::Q_TILE)) >> 4);
         const uint64_t db = dKV + (uint64_t)((st * C::KV_TILE) >> 4);
-        const uint32_t dt = tmem + (uint32_t)(C::BN * t);
+        const uint32_t dt = tmem + (uint32_t)(C::S_STRIDE * t);
         eta_static_for<C::QK_STEPS>([&](auto kk_c) {
           constexpr int kk = decltype(kk_c)::value;
           constexpr uint32_t a_off = ((uint32_t)(kk >> 2) * C::Q_CHUNK + (uint32_t)(kk & 3) * 32u) >> 4;
@@ -429,18 +441,24 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
       };
       // O_t += P_t V : K-steps of 16 keys = 8 TMEM columns of packed bf16 P, 16 rows (2048 B) of V.
       auto issue_pv = [&](int t, int st, bool acc) {
-        const uint32_t tP = C::ALIAS_P ? tmem + (uint32_t)(C::BN * t) : tmem + C::TM_P + (uint32_t)(C::P_COLS * t);
+        const uint32_t tP = C::ALIAS_P      ? tmem + (uint32_t)(C::S_STRIDE * t)
+                            : C::P_IN_HOLES ? tmem + (uint32_t)(C::S_STRIDE * t + C::BN)
+                                            : tmem + C::TM_P + (uint32_t)(C::P_COLS * t);
         const uint64_t db = dV + (uint64_t)((st * C::KV_TILE) >> 4);
         const uint32_t dt = tmem + C::TM_O + (uint32_t)(C::O_COLS * t);
+        const uint32_t tP2 = dt + (uint32_t)D;  // (P_IN_HOLES) keys [64, 96): O_t's spare columns
         const uint32_t acc0 = acc ? 1u : 0u;
         // K-step kk: PV_KEYS keys = 8 TMEM columns of P, PV_KEYS rows (PV_KEYS * 128 B) of V
         eta_static_for<C::BN / C::PV_KEYS>([&](auto kk_c) {
           constexpr int kk = decltype(kk_c)::value;
-          constexpr uint32_t ta_off = 8u * kk, b_off = (uint32_t)(C::PV_KEYS * 128 * kk) / 16u;
-          if constexpr (F8)
-            mma_ts_off_f8<ta_off, b_off>(dt, tP, db, ID_PV, kk > 0 ? 1u : acc0);
-          else
-            mma_ts_off<ta_off, b_off>(dt, tP, db, ID_PV, kk > 0 ? 1u : acc0);
+          constexpr uint32_t b_off = (uint32_t)(C::PV_KEYS * 128 * kk) / 16u;
+          if constexpr (F8) {
+            mma_ts_off_f8<8u * kk, b_off>(dt, tP, db, ID_PV, kk > 0 ? 1u : acc0);
+          } else if constexpr (C::P_IN_HOLES && kk >= 4) {
+            mma_ts_off<8u * (kk - 4), b_off>(dt, tP2, db, ID_PV, 1u);
+          } else {
+            mma_ts_off<8u * kk, b_off>(dt, tP, db, ID_PV, kk > 0 ? 1u : acc0);
+          }
         });
       };
       // Counts over all items; each gives the phase of the barrier it tracks.  With one issuer per tile
@@ -690,9 +708,11 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
   const int row = quarter * 32 + lane;
   const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
   constexpr int BN = C::BN;
-  const uint32_t tS = tmem + lane_addr + (uint32_t)(BN * t);
+  const uint32_t tS = tmem + lane_addr + (uint32_t)(C::S_STRIDE * t);
   const uint32_t tO = tmem + lane_addr + C::TM_O + (uint32_t)(C::O_COLS * t);
-  const uint32_t tP = C::ALIAS_P ? tS : tmem + lane_addr + C::TM_P + (uint32_t)(C::P_COLS * t);
+  const uint32_t tP = C::ALIAS_P      ? tS
+                      : C::P_IN_HOLES ? tS + (uint32_t)BN  // (and O_t's spare columns for keys [64, 96))
+                                      : tmem + lane_addr + C::TM_P + (uint32_t)(C::P_COLS * t);
   const bool causal = HSTU ? true : (p.causal != 0);
   int gj = 0;  // key tiles of Q tile t processed, over all items (phases of s_full, p_full, pv_done)
   bool ok = true;
@@ -833,8 +853,13 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
           tc_fence_after();
         }
       }
+      if constexpr (C::P_IN_HOLES) {
+        ETA_TMEM_ST_X32(tP, pk);                           // keys [0, 64): S_t's spare columns
+        ETA_TMEM_ST_X16(tO + (uint32_t)D, (pk + 32));      // keys [64, 96): O_t's spare columns
+      } else {
 #pragma unroll
-      for (int cc = 0; cc < C::P_COLS / 32; ++cc) ETA_TMEM_ST_X32(tP + 32u * cc, (pk + 32 * cc));
+        for (int cc = 0; cc < C::P_COLS / 32; ++cc) ETA_TMEM_ST_X32(tP + 32u * cc, (pk + 32 * cc));
+      }
       if constexpr (!HSTU) {
         if (__any_sync(0xffffffffu, resc && j > 0)) {
           const uint64_t f2 = f2pack(f, f);
