@@ -268,9 +268,9 @@ __device__ __forceinline__ void dense_unit_block(const PrefillParams &p, int idx
 
 // Work item `idx`: packed launches take the latest row block of every (sequence, head) first; dense ones go
 // group by group (dense_unit_block).
-template <int D, int MODE>
+template <int D, int MODE, bool F8>
 __device__ __forceinline__ PfItem decode_item(const PrefillParams &p, int idx) {
-  constexpr int BN = PfCfg<D>::BN;
+  constexpr int BN = PfCfg<D, F8>::BN;  // the key-tile size of the kernel instance that runs the item
   PfItem it{};
   int half = -1;
   if (idx >= p.n_whole) {  // split halves (only softmax launches with rows > 128 have any)
@@ -350,7 +350,7 @@ __device__ __forceinline__ void prefill_control(const CUtensorMap &tmQ, const CU
             retire();
             break;
           }
-          it = decode_item<D, MODE>(p, (int)idx);
+          it = decode_item<D, MODE, F8>(p, (int)idx);
           if (it.r0 < it.L) break;  // row blocks past the end of their sequence have no work
         }
         ok = mbar_wait(sm.item_empty(k & 1), ((k >> 1) & 1) ^ 1, sm.abort_flag(), p.wait_ns);
