@@ -144,20 +144,22 @@ def test_cu_seqlens_checked_against_T_total(kind, d, tail):
     assert torch.all(lse.cpu()[untouched] == SENTINEL), "lse rows outside the computed sequences were written"
 
 
+@pytest.mark.parametrize("d", [64, 96])
 @pytest.mark.parametrize("big_rows", [False, True])
-def test_hstu_tanh_on_both_pipes(big_rows):
-    """At d = 64 the HSTU tanh of 3 in every 8 pairs runs on the FMA pipe (a polynomial valid for |y| <= 1,
-    y = alpha s / 2) when every row of a warp stays in that range, else the warp keeps every tanh on the
-    MUFU.  With alpha = 1/8 and N(0, 0.5^2) inputs every warp takes the mixed loop; with big_rows the query
-    rows 300..599 of the first sequence are scaled by 8 (exact in bf16), so |y| reaches ~4 there and those
-    warps -- and the rows of warps straddling the boundary -- take the MUFU loop in the same launch."""
+def test_hstu_tanh_on_both_pipes(big_rows, d):
+    """At d = 64 and 96 the HSTU tanh of 3 in every 8 pairs runs on the FMA pipe (a polynomial valid for
+    |y| <= 1, y = alpha s / 2) when every row of a warp stays in that range, else the warp keeps every tanh on
+    the MUFU.  With alpha = 1/8 and N(0, 0.5^2) inputs every warp takes the mixed loop (|y| stays below ~0.6
+    at d = 96); with big_rows the query rows 300..599 of the first sequence are scaled by 8 (exact in
+    bf16), so |y| reaches ~4 there and those warps -- and the rows of warps straddling the boundary -- take
+    the MUFU loop in the same launch."""
     lens = [700, 260]
     cu = inputs.cu_seqlens(lens)
-    T, H, d = int(cu[-1]), 2, 64
+    T, H = int(cu[-1]), 2
     q, k, v = (t.to(DEV) for t in inputs.jagged_qkv(17, T, H, d, std=0.5))
     if big_rows:
         q[300:600] = (q[300:600].float() * 8).to(torch.bfloat16)
     o = eta.hstu_fwd_jagged(q, k, v, cu.to(DEV), max(lens), 0.125, 1.0 / 256)
     assert eta.status() == 0
     o_ref = oracle.hstu_jagged(q, k, v, cu, 0.125, 1.0 / 256)
-    check_hstu(o, o_ref, f"hstu tanh pipes big_rows={big_rows}")
+    check_hstu(o, o_ref, f"hstu tanh pipes d={d} big_rows={big_rows}")
