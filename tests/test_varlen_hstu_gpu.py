@@ -149,7 +149,7 @@ def test_cu_seqlens_checked_against_T_total(kind, d, tail):
 def test_hstu_tanh_on_both_pipes(big_rows, d):
     """At d = 64 and 96 the HSTU tanh of 3 in every 8 pairs runs on the FMA pipe (a polynomial valid for
     |y| <= 1, y = alpha s / 2) when every row of a warp stays in that range, else the warp keeps every tanh on
-    the MUFU.  With alpha = 1/8 and N(0, 0.5^2) inputs every warp takes the mixed loop (|y| stays below ~0.6
+    the MUFU.  With alpha = 1/8 and N(0, 0.5^2) inputs every warp takes the mixed loop (|y| stays below ~0.7
     at d = 96); with big_rows the query rows 300..599 of the first sequence are scaled by 8 (exact in
     bf16), so |y| reaches ~4 there and those warps -- and the rows of warps straddling the boundary -- take
     the MUFU loop in the same launch."""
