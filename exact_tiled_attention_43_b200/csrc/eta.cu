@@ -319,7 +319,7 @@ int prefill_common(int mode, const void *q, const void *k, const void *v, void *
   p.o_f32 = (o_dtype == ETA_OUT_F32);
   p.scale_log2 = scale * qk_descale * 1.4426950408889634f;
   p.hstu_half_alpha = 0.5f * alpha;
-  p.hstu_out = 0.5f * alpha * inv_n;
+  p.hstu_inv_n = inv_n;
   p.o_scale = v_descale;
   p.wait_ns = g_wait_ns;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

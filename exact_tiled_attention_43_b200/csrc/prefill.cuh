@@ -100,7 +100,7 @@ struct PrefillParams {
   int causal, o_f32;
   float scale_log2;        // softmax: scale * log2(e)
   float hstu_half_alpha;   // HSTU: 0.5 * alpha      (tanh argument scale)
-  float hstu_out;          // HSTU: 0.5 * alpha * inv_n
+  float hstu_inv_n;        // HSTU: inv_n (applied to O at the end of an item)
   float o_scale;           // multiplies O / l (1; the V descale factor for e4m3 inputs)
   long long wait_ns;
 };
@@ -799,15 +799,16 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
         rowsum = (r0a + r1a) + (r2a + r3a);
         f = resc ? ex2_approx(m_used - msub) : 1.f;  // 0 on the first tile
       } else {
-        // HSTU: p = inv_n * silu(alpha s) = h + h * tanh(alpha s / 2),  h = (alpha * inv_n / 2) s.
-        // Masked keys get s = 0 first, which gives p = 0 exactly (h = 0), so the pointwise loop is the same
-        // straight-line code for every tile.
+        // HSTU: p = inv_n * silu(alpha s) = inv_n (y + y tanh(y)),  y = alpha s / 2.  P holds y + y tanh(y)
+        // and the factor inv_n is applied to O at the end of the item (one multiply a row instead of one a
+        // score).  Masked keys get s = 0 first, which gives p = 0 exactly (y = 0), so the pointwise loop is
+        // the same straight-line code for every tile.
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
             if (c > kmax) sr[c] = 0u;
         }
-        const uint64_t ha2 = f2pack(p.hstu_half_alpha, p.hstu_half_alpha), ho2 = f2pack(p.hstu_out, p.hstu_out);
+        const uint64_t ha2 = f2pack(p.hstu_half_alpha, p.hstu_half_alpha);
         // tanh on the MUFU for every pair, or (TANH_FMA_PAIRS of every 8 pairs) on the FMA pipe by the degree-7
         // polynomial, so that the two pipes share the work.  The polynomial holds for |alpha s / 2| <= 1: a
         // warp takes the mixed loop only when every row's polynomial pairs are in that range.
@@ -825,7 +826,6 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
           for (int i = 0; i < BN / 2; ++i) {
             const uint64_t s2 = f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
             const uint64_t y2 = mul_x2(s2, ha2);
-            const uint64_t h2 = mul_x2(s2, ho2);
             uint64_t t2;
             if (decltype(with_poly)::value && (i % 8) < C::TANH_FMA_PAIRS) {
               t2 = tanh_poly_x2(y2);
@@ -835,7 +835,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
               t2 = f2pack(tanh_approx(y0), tanh_approx(y1));
             }
             float p0, p1;
-            f2unpack(fma_x2(h2, t2, h2), p0, p1);
+            f2unpack(fma_x2(y2, t2, y2), p0, p1);
             pk[i] = pack_bf16x2(p0, p1);
           }
         };
@@ -917,7 +917,7 @@ __device__ __forceinline__ void prefill_softmax(const PrefillParams &p, uint8_t 
         merge = true;
       }
     }
-    const float inv_l = HSTU ? 1.f : ((l_fin > 0.f) ? p.o_scale / l_fin : 0.f);
+    const float inv_l = HSTU ? p.hstu_inv_n : ((l_fin > 0.f) ? p.o_scale / l_fin : 0.f);
     const float w0 = a0 * inv_l, w1 = a1 * inv_l;
     const bool valid = qpos < L;
     const uint32_t tO1 = tmem + lane_addr + C::TM_O + (uint32_t)C::O_COLS;  // O_1 (read here only when merging)
